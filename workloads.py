@@ -1,0 +1,129 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module holds shapes, seeds and random draws only -- none of the
+attention arithmetic.  Both sides of every parity check (the float64 oracle
+and the CUDA library) read tensors made here, so a result never depends on
+which side generated its own inputs.
+
+Recipe: a ``torch.Generator`` seeded with the workload's seed draws, in order,
+q, k, v (and dO for the backward) as float32 standard normals, which are then
+rounded to the workload's dtype.  The decode workload first draws its
+per-sequence cache lengths from a CPU generator (uniform integers in
+[lo, hi]), then q and the two caches.  Draws on a CUDA device use torch's CUDA
+generator with the same seed; those values differ from the CPU stream, which
+does not matter because both sides read the same tensors.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+BF16 = torch.bfloat16
+FP32 = torch.float32
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One named attention workload (shapes, masks, dtype, seed)."""
+
+    name: str
+    kind: str            # "forward", "decode" or "forward_backward"
+    B: int
+    H: int
+    N: int               # sequence length (decode: cache capacity)
+    d: int
+    dtype: torch.dtype
+    seed: int
+    causal: bool = False
+    window: int = 0
+    seqlen_lo: int = 0   # decode only: per-sequence cache length range
+    seqlen_hi: int = 0
+    notes: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("single_head_fp32", "forward", 1, 1, 128, 64, FP32, 0,
+                 notes="single-head fp32 forward, non-causal"),
+        Workload("causal_prefill", "forward", 4, 16, 2048, 128, BF16, 1, causal=True,
+                 notes="causal prefill forward, bf16 in / fp32 accumulate"),
+        Workload("sliding_window_long", "forward", 1, 32, 16384, 128, BF16, 2,
+                 causal=True, window=4096,
+                 notes="long-context causal sliding window (i-4096 < j <= i)"),
+        Workload("kv_cache_decode", "decode", 64, 32, 8192, 128, BF16, 3,
+                 seqlen_lo=512, seqlen_hi=8192,
+                 notes="single-token decode, padded cache capacity 8192"),
+        Workload("causal_fwd_bwd", "forward_backward", 2, 16, 4096, 128, BF16, 4,
+                 causal=True, notes="causal forward + recompute backward"),
+    ]
+}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    return g
+
+
+def randn(shape, dtype, gen: torch.Generator, device) -> torch.Tensor:
+    """float32 N(0,1) draw rounded to ``dtype`` (round-to-nearest-even)."""
+    return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(dtype)
+
+
+def forward_inputs(B, H, N, d, dtype=BF16, seed=0, device="cpu", with_dout=False):
+    """q, k, v (and dO) of shape [B, H, N, d], contiguous, i.i.d. N(0,1)."""
+    g = _gen(seed, device)
+    q = randn((B, H, N, d), dtype, g, device)
+    k = randn((B, H, N, d), dtype, g, device)
+    v = randn((B, H, N, d), dtype, g, device)
+    if with_dout:
+        dO = randn((B, H, N, d), dtype, g, device)
+        return q, k, v, dO
+    return q, k, v
+
+
+def decode_seqlens(B, lo, hi, seed) -> torch.Tensor:
+    """Per-sequence cache lengths, uniform integers in [lo, hi] (int32, CPU)."""
+    g = _gen(seed, "cpu")
+    return torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+def decode_inputs(B, H, cap, d, lo, hi, dtype=BF16, seed=0, device="cpu",
+                  pad_value: float | None = None):
+    """q [B,H,d], kcache/vcache [B,H,cap,d], seqlens [B] (int32, on ``device``).
+
+    Cache rows at positions >= seqlens[b] are also random unless ``pad_value``
+    is given, in which case they are filled with it (NaN makes any read past a
+    sequence's length visible in the output).
+    """
+    seqlens = decode_seqlens(B, lo, hi, seed)
+    g = _gen(seed, device)
+    q = randn((B, H, d), dtype, g, device)
+    kc = torch.empty((B, H, cap, d), dtype=dtype, device=device)
+    vc = torch.empty((B, H, cap, d), dtype=dtype, device=device)
+    for b in range(B):  # per sequence, to bound the float32 staging buffer
+        kc[b] = randn((H, cap, d), dtype, g, device)
+        vc[b] = randn((H, cap, d), dtype, g, device)
+    if pad_value is not None:
+        for b in range(B):
+            n = int(seqlens[b])
+            kc[b, :, n:] = pad_value
+            vc[b, :, n:] = pad_value
+    return q, kc, vc, seqlens.to(device)
+
+
+def workload_inputs(w: Workload, device="cpu", **kw):
+    """Inputs of a named workload at its full size."""
+    if w.kind == "decode":
+        return decode_inputs(w.B, w.H, w.N, w.d, w.seqlen_lo, w.seqlen_hi, w.dtype,
+                             w.seed, device, **kw)
+    return forward_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed, device,
+                          with_dout=(w.kind == "forward_backward"))
+
