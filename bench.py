@@ -1,0 +1,429 @@
+"""Benchmark of the tiled exact attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the hot path over one batch of synthetic input:
+  causal_prefill (default): fa_forward on B=4, H=16, N=2048, d=128, bf16, causal
+  sliding_window_long:      fa_forward on B=1, H=32, N=16384, d=128, window 4096
+  kv_cache_decode:          fa_decode, batch 64 x 32 heads, cache lengths U[512, 8192]
+  causal_fwd_bwd:           fa_forward + fa_backward on B=2, H=16, N=4096, d=128
+Inputs are seeded N(0,1) draws (``workloads.py``), resident in HBM before the
+timed region.  The L2 (126 MB) is flushed between timed steps by writing a
+256 MiB buffer outside the timed events.  Throughput counts only the (query,
+key) pairs the mask allows: 4*d FLOPs per pair forward, 10*d backward;
+decode counts the bytes of the K/V rows it must read plus q and o.
+
+Prints one JSON line (rank 0).  With --gpus N > 1 (launched by torchrun) each
+rank runs its own independent batch (weak scaling, no collective on the data
+path); value = all ranks' work / the slowest rank's time.
+
+--impl reference times the float64 CPU oracle (the only other
+implementation of this method) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+_CPU_THREADS = str(os.cpu_count() or 1)
+for _v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+    os.environ.setdefault(_v, _CPU_THREADS)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- work counts
+def allowed_pairs(N: int, causal: bool, window: int) -> int:
+    """(query, key) pairs one head's mask allows, in closed form per row."""
+    i = np.arange(N, dtype=np.int64)
+    hi = i + 1 if causal else np.full(N, N, dtype=np.int64)
+    lo = np.maximum(0, i - window + 1) if window > 0 else np.zeros(N, dtype=np.int64)
+    return int(np.maximum(0, hi - lo).sum())
+
+
+def forward_flops(w) -> float:
+    return 4.0 * w.d * allowed_pairs(w.N, w.causal, w.window) * w.B * w.H
+
+
+def backward_flops(w) -> float:
+    return 10.0 * w.d * allowed_pairs(w.N, w.causal, w.window) * w.B * w.H
+
+
+def decode_bytes(w, seqlens) -> float:
+    rows = float(np.minimum(np.asarray(seqlens, dtype=np.int64), w.N).sum()) * w.H
+    return rows * w.d * 2 * 2 + 2 * w.B * w.H * w.d * 2  # K + V rows, q + o
+
+
+# ----------------------------------------------------------------------------- measurement helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def source_hash(names):
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_exact_attention_forward_b200", "csrc")
+    for n in sorted(names):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, sources):
+    """DRAM bytes per launch from the committed ncu summary, if it is current."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != source_hash(sources):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        smax = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.5 * smax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, s in enumerate(r[2]) if s.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in loaded])), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        n = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        return int(max(n)) if n else int(_CPU_THREADS)
+    except Exception:  # noqa: BLE001
+        return int(_CPU_THREADS)
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+def oracle_sample(w, budget_s=12.0):
+    """Time the float64 oracle on whole heads of the workload until ~budget_s.
+
+    Returns (value in the workload's unit, sample description)."""
+    import oracle
+
+    gen = torch.Generator().manual_seed(w.seed)
+    t_total, units, heads = 0.0, 0.0, 0
+    while t_total < budget_s and heads < w.B * w.H:
+        if w.kind == "decode":
+            n = int(workloads.decode_seqlens(w.B, w.seqlen_lo, w.seqlen_hi, w.seed)[heads % w.B])
+            q = torch.randn(1, 1, w.d, generator=gen).to(w.dtype)
+            kc = torch.randn(1, 1, n, w.d, generator=gen).to(w.dtype)
+            vc = torch.randn(1, 1, n, w.d, generator=gen).to(w.dtype)
+            t0 = time.perf_counter()
+            oracle.decode_forward(q, kc, vc, np.array([n]), w.scale)
+            t_total += time.perf_counter() - t0
+            units += n * w.d * 2 * 2 + 2 * w.d * 2
+        else:
+            q, k, v = (torch.randn(w.N, w.d, generator=gen).to(w.dtype) for _ in range(3))
+            t0 = time.perf_counter()
+            o, lse = oracle.attention_forward(q, k, v, w.scale, w.causal, w.window)
+            if w.kind == "forward_backward":
+                oracle.attention_backward(q, k, v, torch.randn(w.N, w.d, generator=gen).to(w.dtype),
+                                          w.scale, w.causal, w.window)
+            t_total += time.perf_counter() - t0
+            per = 4.0 * w.d * allowed_pairs(w.N, w.causal, w.window)
+            if w.kind == "forward_backward":
+                per *= 3.5
+            units += per
+        heads += 1
+    rate = units / t_total
+    if w.kind == "decode":
+        return rate / 1e9, f"{heads} of {w.B * w.H} (sequence, head) decodes, {t_total:.1f} s"
+    return rate / 1e12, f"{heads} of {w.B * w.H} heads (full N x N float64 per head), {t_total:.1f} s"
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def make_step(w, dev):
+    """Returns (step_fn, e2e_fn, units_per_step, unit, metric, launches_per_step, kernel, sources)."""
+    import tiled_exact_attention_forward_b200 as fa
+
+    if w.kind == "decode":
+        q, kc, vc, seqlens = workloads.workload_inputs(w, device=dev)
+        ws = torch.empty(fa.decode_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
+        units = decode_bytes(w, seqlens.cpu().numpy()) / 1e9
+
+        def step():
+            fa.decode(q, kc, vc, seqlens, w.scale, workspace=ws, out=o, lse=lse)
+
+        # End to end: a decode step's own inputs (the new query and the lengths) go up,
+        # the output comes back; the cache stays resident as it would in serving.
+        q_h = q.cpu().pin_memory()
+        s_h = seqlens.cpu().pin_memory()
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e():
+            q.copy_(q_h, non_blocking=True)
+            seqlens.copy_(s_h, non_blocking=True)
+            fa.decode(q, kc, vc, seqlens, w.scale, workspace=ws, out=o, lse=lse)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        h2d = q_h.numel() * q_h.element_size() + s_h.numel() * 4
+        d2h = o_h.numel() * o_h.element_size() + l_h.numel() * 4
+        return (step, e2e, units, "GB/s", "decode GB/s", 2, "decode_split_kernel",
+                ["decode.cu", "common.cuh", "kernels.h"], h2d, d2h)
+
+    with_bwd = w.kind == "forward_backward"
+    ins = workloads.workload_inputs(w, device=dev)
+    q, k, v = ins[:3]
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flops = forward_flops(w) + (backward_flops(w) if with_bwd else 0.0)
+    if with_bwd:
+        dO = ins[3]
+        ws = torch.empty(fa.backward_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step():
+        fa.forward(q, k, v, w.causal, w.window, w.scale, out=o, lse=lse)
+        if with_bwd:
+            fa.backward(q, k, v, o, dO, lse, w.causal, w.window, w.scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    host_in = [t.cpu().pin_memory() for t in ins]
+    outs = [o, lse] + ([dq, dk, dv] if with_bwd else [])
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+
+    def e2e():
+        for hd, dd in zip(host_in, ins):
+            dd.copy_(hd, non_blocking=True)
+        step()
+        for hd, dd in zip(host_out, outs):
+            hd.copy_(dd, non_blocking=True)
+
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    metric = "attention TFLOP/s (fwd+bwd, unmasked FLOPs)" if with_bwd else \
+        "attention TFLOP/s (fwd, unmasked FLOPs)"
+    return (step, e2e, flops / 1e12, "TFLOP/s", metric, 4 if with_bwd else 1,
+            "bwd_main_kernel" if with_bwd else "fwd_tc_kernel",
+            ["bwd.cu" if with_bwd else "fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
+
+
+def timed_loop(fn, steps, warmup, flush, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        flush.add_(1)  # 256 MiB write: evicts the previous step's data from L2 (not timed)
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def run_gpu(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    import tiled_exact_attention_forward_b200 as fa
+
+    fa.library()
+    w = workloads.WORKLOADS[args.workload]
+    (step, e2e, units, unit, metric, launches, kernel, sources, h2d, d2h) = make_step(w, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        times = timed_loop(step, args.steps, 0, flush, stream)
+    barrier()
+    if fa.device_status(dev) != fa.FA_OK:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    ms = float(np.mean(times))
+    e2e_times = timed_loop(e2e, max(3, args.steps // 2), 2, flush, stream)
+    barrier()
+    e2e_ms = float(np.mean(e2e_times))
+    if dist:
+        t = torch.tensor([ms, e2e_ms], device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    value = units * world / (ms / 1e3)
+    e2e_value = units * world / (e2e_ms / 1e3)
+    hbm, tflops, peak_kind = load_peaks()
+    if unit == "GB/s":
+        roof = {"bound": "hbm", "achieved": units / (ms / 1e3), "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": units / (ms / 1e3), "peak": tflops, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_kind} ({'copy bandwidth' if unit == 'GB/s' else 'cuBLAS bf16 burst'})"
+    roof["kernel"] = kernel
+    roof["traffic"] = profiled_traffic(kernel, sources)
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "window": w.window, "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between timed steps (256 MiB write, untimed)"},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample = oracle_sample(w)
+        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cpu_threads_used(), "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+def run_reference(args):
+    w = workloads.WORKLOADS[args.workload]
+    t0 = time.perf_counter()
+    vals = []
+    samples = []
+    for i in range(args.warmup + args.steps):
+        v, sample = oracle_sample(w, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            vals.append(v)
+            samples.append(sample)
+    unit = "GB/s" if w.kind == "decode" else "TFLOP/s"
+    value = float(np.mean(vals))
+    metric = {"decode": "decode GB/s", "forward_backward": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)"} \
+        .get(w.kind, "attention TFLOP/s (fwd, unmasked FLOPs)")
+    return {
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+                   "window": w.window},
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": unit, "cores": cpu_threads_used(),
+                         "sample": samples[-1] if samples else ""},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="causal_prefill", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=4.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) tiled exact attention library.
+ *
+ * Exact scaled-dot-product attention
+ *     O = softmax(Q K^T * scale + mask) V
+ * computed tile by tile with the online softmax (a running row max m and row
+ * sum l, the output rescaled by exp(m_old - m_new) when the max grows and
+ * divided by l once at the end), so the N x N score matrix never reaches
+ * device memory.  Sources, by page title and section:
+ *   - "Building Flash Attention from Scratch in Pure NumPy": architecture
+ *     overview (per-query-block data flow), Step 2 (online softmax update),
+ *     Step 3 (the forward's tile loops and its scale=None default), Step 4
+ *     (the backward from the saved row statistics, D = rowsum(dO * O)).
+ *   - "Build a FlashAttention-2 Inference Kernel from Scratch in Pure Python":
+ *     Steps 2-3 (scale, mask to -inf, causal j <= i, sliding-window skipping).
+ *   - "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
+ *     Python": Step 4 (single-query decode against a key/value cache).
+ *
+ * Conventions shared by every entry point
+ *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major
+ *     [B][H][N][d] (d innermost).  lse is float32 [B][H][N].  Decode: q and o
+ *     are [B][H][d], the caches [B][H][cap][d], seqlens int32 [B].
+ *   - Mask: key j is visible to query i iff
+ *         (causal == 0 || j <= i) && (window <= 0 || j > i - window),
+ *     so a window holds exactly `window` keys including the query itself.
+ *   - scale <= 0 selects 1/sqrt(d).
+ *   - lse is the natural-log logsumexp of the row's scaled, masked scores.
+ *     A row with no visible key gets O = 0 and lse = -inf.
+ *   - Pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer, including workspaces.  The library allocates no device memory
+ *     and keeps no per-call state.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns without synchronising.
+ *   - Argument errors are found on the host before anything is launched:
+ *     FA_ERR_INVALID (null pointer, non-positive size, misaligned pointer,
+ *     workspace too small, window < 0) or FA_ERR_UNSUPPORTED (a dtype/d
+ *     combination with no kernel).  FA_ERR_CUDA reports a failed launch.
+ *   - Kernels never trap.  A kernel that waits too long on an internal
+ *     barrier records FA_ERR_TIMEOUT in a device status word and returns;
+ *     fa_get_device_status() reports it.
+ */
+#ifndef TILED_EXACT_ATTENTION_FA_H_
+#define TILED_EXACT_ATTENTION_FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status;
+
+typedef enum {
+  FA_BF16 = 0, /* bfloat16 inputs/outputs, float32 accumulation (d = 128)   */
+  FA_FP32 = 1  /* float32 inputs/outputs, float32 arithmetic (d = 64 or 128) */
+} fa_dtype;
+
+/*
+ * Forward pass.  "Building Flash Attention from Scratch in Pure NumPy",
+ * architecture overview and Steps 2-3; masks from "Build a FlashAttention-2
+ * Inference Kernel from Scratch in Pure Python", Step 3.
+ *
+ *   q, k, v : [B][H][N][d] inputs (dtype), 16-byte aligned.
+ *   o       : [B][H][N][d] output (dtype), 16-byte aligned.
+ *   lse     : [B][H][N] float32 output (natural-log logsumexp per row); may
+ *             be NULL when the caller does not need it.
+ *   B, H, N : >= 1.  d: 128 for FA_BF16; 64 or 128 for FA_FP32.
+ *   causal  : 0 or 1.  window: 0 = none, else > 0 (see Mask above).
+ * Key tiles that the mask hides completely are skipped, never computed.
+ * FA_BF16 runs on the tensor cores (tcgen05, TMA, TMEM); FA_FP32 on CUDA
+ * cores in float32.
+ */
+FA_API fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal, int window,
+                     fa_dtype dtype, void* stream);
+
+/*
+ * Bytes of device workspace fa_decode needs for these sizes (a multiple of
+ * 256; 0 for invalid sizes).  The workspace holds one partial (o, lse) per
+ * key chunk of each (b, h) between the split and combine kernels.
+ */
+FA_API size_t fa_decode_workspace_size(int B, int H, int cap, int d);
+
+/*
+ * Single-token decode against a padded key/value cache.  "Build a
+ * FlashAttention Kernel with Online Softmax and KV Cache in Pure Python",
+ * Step 4: the cache already holds the current token, so query (b, h) attends
+ * to every cached position j < seqlens[b].  The keys are split into chunks
+ * scored in parallel; the chunk results are merged with the two-softmax merge
+ * identity from "Building Flash Attention from Scratch in Pure NumPy"
+ * (architecture overview): lse = ln sum_s exp(lse_s), O = sum_s
+ * exp(lse_s - lse) O_s.
+ *
+ *   q        : [B][H][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   kcache,
+ *   vcache   : [B][H][cap][d], 16-byte aligned.  Rows at j >= seqlens[b]
+ *              are never read.
+ *   seqlens  : [B] int32 DEVICE array.  Values are clamped to [0, cap]; a
+ *              length of 0 gives o = 0, lse = -inf.
+ *   o        : [B][H][d] output (dtype).  lse: [B][H] float32 or NULL.
+ *   workspace: >= fa_decode_workspace_size(B, H, cap, d) bytes, 256-byte
+ *              aligned, contents ignored on entry.
+ */
+FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache,
+                    const int32_t* seqlens, void* o, float* lse,
+                    int B, int H, int cap, int d, float scale, fa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Bytes of device workspace fa_backward needs (a multiple of 256): the
+ * float32 row terms D = rowsum(dO * O) and a float32 dQ accumulator.
+ */
+FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass.  "Building Flash Attention from Scratch in Pure NumPy",
+ * Step 4: D = rowsum(dO * O); per key tile, P is recomputed from the saved
+ * row statistic (here the single logsumexp lse written by fa_forward) and
+ *     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+ *     dQ = scale * dS K,  dK = scale * dS^T Q
+ * (that page's own dK/dQ lines are declared simplified; these are the exact
+ * gradients of the forward).
+ *
+ *   q, k, v, o, dout : [B][H][N][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   lse              : [B][H][N] float32 from fa_forward with the same
+ *                      arguments.
+ *   dq, dk, dv       : [B][H][N][d] outputs (dtype).
+ *   workspace        : >= fa_backward_workspace_size(B, H, N, d) bytes,
+ *                      256-byte aligned, contents ignored on entry.
+ */
+FA_API fa_status fa_backward(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      int B, int H, int N, int d, float scale, int causal, int window,
+                      fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns FA_ERR_TIMEOUT if any kernel of this
+ * library recorded a barrier timeout since the last call (and clears the
+ * record), FA_ERR_CUDA if the stream reports an error, else FA_OK.
+ */
+FA_API fa_status fa_get_device_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+FA_API const char* fa_status_string(fa_status status);
+
+/* Library ABI version (major * 100 + minor). */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILED_EXACT_ATTENTION_FA_H_ */

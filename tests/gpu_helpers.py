@@ -1,0 +1,50 @@
+"""Shared pieces of the GPU parity tests: tolerances and comparisons.
+
+Tolerances (fixed by the task's stated bar, written here once):
+  forward / decode outputs: max |err| <= 2e-2 and mean |err| <= 2e-3
+  logsumexp:                max |err| <= 1e-3
+  gradients:                max |err| <= 5e-2 * max |reference gradient|
+  float32 forward:          max |err| <= 1e-4 (the NumPy page's allclose atol)
+"""
+import numpy as np
+import pytest
+import torch
+
+OUT_MAX = 2e-2
+OUT_MEAN = 2e-3
+LSE_MAX = 1e-3
+GRAD_REL = 5e-2
+FP32_ATOL = 1e-4
+
+requires_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def to64(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        return t.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+def assert_output_close(got, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN):
+    got, ref = to64(got), to64(ref)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - ref)
+    assert err.max() <= max_tol, f"{what}: max |err| {err.max():.3g} > {max_tol}"
+    assert err.mean() <= mean_tol, f"{what}: mean |err| {err.mean():.3g} > {mean_tol}"
+
+
+def assert_lse_close(got, ref, what, tol=LSE_MAX):
+    got, ref = to64(got), to64(ref)
+    both_inf = np.isneginf(got) & np.isneginf(ref)
+    err = np.abs(np.where(both_inf, 0.0, got - ref))
+    assert np.all(np.isfinite(err)), f"{what}: lse mismatch in -inf pattern"
+    assert err.max() <= tol, f"{what}: lse max |err| {err.max():.3g} > {tol}"
+
+
+def assert_grad_close(got, ref, what, rel=GRAD_REL):
+    got, ref = to64(got), to64(ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    scale = max(np.abs(ref).max(), 1e-30)
+    err = np.abs(got - ref).max()
+    assert err <= rel * scale, f"{what}: max |err| {err:.3g} > {rel} * {scale:.3g}"

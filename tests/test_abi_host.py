@@ -1,0 +1,108 @@
+"""The C ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tiled_exact_attention_forward_b200 as fa
+from tiled_exact_attention_forward_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return fa.library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert set(names) == set(fa.EXPORTED_SYMBOLS), names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    for code in range(5):
+        assert lib.fa_status_string(code).startswith(b"FA_")
+    assert lib.fa_status_string(99) == b"unknown fa_status"
+    assert lib.fa_version() == 100
+
+
+P = ctypes.c_void_p
+GOOD = P(0x100000)       # 16-byte aligned, never dereferenced: validation fails first
+MISALIGNED = P(0x100008)
+
+
+def fwd(lib, q=GOOD, k=GOOD, v=GOOD, o=GOOD, lse=None, B=1, H=1, N=128, d=128, causal=0,
+        window=0, dtype=fa.FA_BF16):
+    return lib.fa_forward(q, k, v, o, lse, B, H, N, d, 0.0, causal, window, dtype, None)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    assert fwd(lib, q=None) == fa.FA_ERR_INVALID
+    assert fwd(lib, o=None) == fa.FA_ERR_INVALID
+    assert fwd(lib, B=0) == fa.FA_ERR_INVALID
+    assert fwd(lib, H=-1) == fa.FA_ERR_INVALID
+    assert fwd(lib, N=0) == fa.FA_ERR_INVALID
+    assert fwd(lib, window=-1) == fa.FA_ERR_INVALID
+    assert fwd(lib, causal=2) == fa.FA_ERR_INVALID
+    assert fwd(lib, k=MISALIGNED) == fa.FA_ERR_INVALID
+    assert fwd(lib, lse=P(0x100002)) == fa.FA_ERR_INVALID
+    assert fwd(lib, d=64) == fa.FA_ERR_UNSUPPORTED          # bf16 needs d = 128
+    assert fwd(lib, d=96, dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
+    assert fwd(lib, dtype=7) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments(lib):
+    ws = lib.fa_decode_workspace_size(2, 3, 1000, 128)
+    assert ws > 0 and ws % 256 == 0
+    assert lib.fa_decode_workspace_size(0, 3, 1000, 128) == 0
+
+    def dec(q=GOOD, seqlens=GOOD, ws_ptr=GOOD, ws_bytes=ws, cap=1000, d=128, dtype=fa.FA_BF16):
+        return lib.fa_decode(q, GOOD, GOOD, seqlens, GOOD, None, 2, 3, cap, d, 0.0, dtype,
+                             ws_ptr, ws_bytes, None)
+
+    assert dec(q=None) == fa.FA_ERR_INVALID
+    assert dec(seqlens=None) == fa.FA_ERR_INVALID
+    assert dec(ws_ptr=None) == fa.FA_ERR_INVALID
+    assert dec(ws_ptr=P(0x100010)) == fa.FA_ERR_INVALID      # workspace must be 256-aligned
+    assert dec(ws_bytes=ws - 1) == fa.FA_ERR_INVALID
+    assert dec(cap=0) == fa.FA_ERR_INVALID
+    assert dec(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert dec(dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments(lib):
+    ws = lib.fa_backward_workspace_size(1, 2, 300, 128)
+    assert ws >= (2 * 300 * 4) + (2 * 300 * 128 * 4) and ws % 256 == 0
+
+    def bwd(lse=GOOD, ws_ptr=GOOD, ws_bytes=ws, N=300, d=128, window=0):
+        return lib.fa_backward(GOOD, GOOD, GOOD, GOOD, GOOD, lse, GOOD, GOOD, GOOD, 1, 2, N, d,
+                               0.0, 1, window, fa.FA_BF16, ws_ptr, ws_bytes, None)
+
+    assert bwd(lse=None) == fa.FA_ERR_INVALID
+    assert bwd(ws_bytes=ws - 256) == fa.FA_ERR_INVALID
+    assert bwd(ws_ptr=None) == fa.FA_ERR_INVALID
+    assert bwd(window=-3) == fa.FA_ERR_INVALID
+    assert bwd(N=0) == fa.FA_ERR_INVALID
+    assert bwd(d=64) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+
+    q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)

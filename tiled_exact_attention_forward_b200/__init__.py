@@ -1,0 +1,221 @@
+"""B200 (sm_100a) tiled exact attention: a thin ctypes binding over libfa_b200.so.
+
+Every step of the computation runs in the CUDA library's kernels; this module
+only checks tensor shapes, allocates outputs and workspaces with torch, and
+passes raw device pointers and the current CUDA stream to the C ABI declared
+in ``include/fa.h``.  There is no CPU fallback: if the library or a CUDA
+device is missing, calls raise.
+
+Functions (names follow the C ABI):
+    forward(q, k, v, causal=False, window=0, scale=None)        -> (o, lse)
+    decode(q, kcache, vcache, seqlens, scale=None)               -> (o, lse)
+    backward(q, k, v, o, dout, lse, causal=False, window=0,
+             scale=None)                                         -> (dq, dk, dv)
+    forward_host(...)  -- forward on pinned host tensors (copies in and out)
+    device_status()    -- FA_OK or the first recorded device-side timeout
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_BF16, FA_FP32 = 0, 1
+
+EXPORTED_SYMBOLS = (
+    "fa_forward",
+    "fa_decode_workspace_size",
+    "fa_decode",
+    "fa_backward_workspace_size",
+    "fa_backward",
+    "fa_get_device_status",
+    "fa_status_string",
+    "fa_version",
+)
+
+
+class FAError(RuntimeError):
+    """A non-FA_OK status from the C ABI."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib().fa_status_string(status).decode() if _LIB is not None else str(status)
+        super().__init__(f"{where}: {msg}")
+
+
+_LIB = None
+
+
+def _lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m tiled_exact_attention_forward_b200.build`"
+        )
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_forward.argtypes = [P, P, P, P, P, I, I, I, I, F, I, I, I, P]
+    lib.fa_forward.restype = I
+    lib.fa_decode_workspace_size.argtypes = [I, I, I, I]
+    lib.fa_decode_workspace_size.restype = Z
+    lib.fa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
+    lib.fa_decode.restype = I
+    lib.fa_backward_workspace_size.argtypes = [I, I, I, I]
+    lib.fa_backward_workspace_size.restype = Z
+    lib.fa_backward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, I, I, P, Z, P]
+    lib.fa_backward.restype = I
+    lib.fa_get_device_status.argtypes = [P]
+    lib.fa_get_device_status.restype = I
+    lib.fa_status_string.argtypes = [I]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_version.argtypes = []
+    lib.fa_version.restype = I
+    _LIB = lib
+    return lib
+
+
+def library() -> ctypes.CDLL:
+    """The loaded C library (raises ImportError if it has not been built)."""
+    return _lib()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != FA_OK:
+        raise FAError(status, where)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return FA_BF16
+    if dt == torch.float32:
+        return FA_FP32
+    raise TypeError(f"unsupported dtype {dt}: use torch.bfloat16 or torch.float32")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _scale_arg(scale) -> float:
+    return 0.0 if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, window: int = 0, scale=None, out=None, lse=None):
+    """O = softmax(q k^T * scale + mask) v and the float32 row logsumexp.
+
+    q, k, v: [B, H, N, d] contiguous CUDA tensors (bf16 with d = 128, or fp32
+    with d in {64, 128}).  Returns (o, lse) with o like q and lse [B, H, N].
+    """
+    _need_cuda(q, k, v)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    o = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    st = _lib().fa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d,
+                           _scale_arg(scale), int(bool(causal)), int(window),
+                           _dtype_code(q.dtype), _stream(q.device))
+    _check(st, "fa_forward")
+    return o, lse
+
+
+def forward_host(q, k, v, causal: bool = False, window: int = 0, scale=None, device="cuda"):
+    """The forward for host tensors: copy in (pinned -> device), run, copy out.
+
+    Returns host (o, lse).  The copies are ordered on the current stream.
+    """
+    dev = torch.device(device)
+    qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    o, lse = forward(qd, kd, vd, causal, window, scale)
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    o_h.copy_(o, non_blocking=True)
+    l_h.copy_(lse, non_blocking=True)
+    torch.cuda.current_stream(dev).synchronize()
+    return o_h, l_h
+
+
+def decode_workspace_size(B, H, cap, d) -> int:
+    return int(_lib().fa_decode_workspace_size(B, H, cap, d))
+
+
+def decode(q, kcache, vcache, seqlens, scale=None, workspace=None, out=None, lse=None):
+    """Single-token decode: q [B, H, d] against kcache/vcache [B, H, cap, d].
+
+    seqlens: int32 [B] CUDA tensor; query (b, h) attends to cache rows
+    j < seqlens[b].  Returns (o [B, H, d] bf16, lse [B, H] float32).
+    """
+    _need_cuda(q, kcache, vcache, seqlens)
+    B, H, d = q.shape
+    cap = kcache.shape[2]
+    if kcache.shape != (B, H, cap, d) or vcache.shape != kcache.shape:
+        raise ValueError("kcache/vcache must be [B, H, cap, d] matching q")
+    if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
+        raise ValueError("seqlens must be an int32 tensor of shape [B]")
+    need = decode_workspace_size(B, H, cap, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = _lib().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse),
+                          B, H, cap, d, _scale_arg(scale), _dtype_code(q.dtype),
+                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(q.device))
+    _check(st, "fa_decode")
+    return o, lse
+
+
+def backward_workspace_size(B, H, N, d) -> int:
+    return int(_lib().fa_backward_workspace_size(B, H, N, d))
+
+
+def backward(q, k, v, o, dout, lse, causal: bool = False, window: int = 0, scale=None,
+             workspace=None, dq=None, dk=None, dv=None):
+    """Gradients (dq, dk, dv) of the forward, recomputing P from lse."""
+    _need_cuda(q, k, v, o, dout, lse)
+    B, H, N, d = q.shape
+    for t in (k, v, o, dout):
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k, v, o, dout must share shape and dtype")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 [B, H, N]")
+    need = backward_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = _lib().fa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                            _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale_arg(scale),
+                            int(bool(causal)), int(window), _dtype_code(q.dtype),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(q.device))
+    _check(st, "fa_backward")
+    return dq, dk, dv
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return the library's device status."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(_lib().fa_get_device_status(_stream(dev)))

@@ -1,0 +1,473 @@
+// Backward pass (bf16, d = 128) on the tensor cores.
+//
+// "Building Flash Attention from Scratch in Pure NumPy", Step 4: precompute
+// D = rowsum(dO * O); then for each key tile, loop over the query tiles that
+// can see it, recompute the probabilities from the saved row statistic and
+// accumulate the gradients.  That page's own dK/dQ lines are declared
+// simplified; the exact gradients of the forward are used instead:
+//     P = exp(S * scale - lse),  dV += P^T dO,  dP = dO V^T,
+//     dS = P * (dP - D),  dK += scale * dS^T Q,  dQ += scale * dS K.
+//
+// Kernels: bwd_pre (D and zeroed fp32 dQ accumulator), bwd_main (below),
+// bwd_post (dQ fp32 -> bf16).
+//
+// bwd_main, one CTA per (batch*head, 128-key tile), 320 threads:
+//   * warp 9 loads K and V once, then (Q_i, dO_i) pairs by TMA into a
+//     two-stage ring;
+//   * warp 8 allocates tensor memory and issues the MMAs from one thread;
+//   * warps 0-3 (one thread per key row = one TMEM lane) turn S^T, dP^T into
+//     P^T and dS^T: bf16 back into tensor memory (operands of the dV and dK
+//     MMAs) and dS^T into shared memory (operand of the dQ MMA);
+//   * warps 4-7 (one thread per query row) read dQ_i out of tensor memory
+//     and add it into the fp32 accumulator with vector reductions; at the
+//     end warps 0-3 write dV and warps 4-7 write dK.
+// Tensor memory (512 columns): [S^T -> P^T, later dQ_i] [dP^T -> dS^T] [dV] [dK].
+// Keys are the MMA rows of S^T = K Q^T and dP^T = V dO^T, so P^T and dS^T
+// land with keys on lanes -- exactly the A operands dV and dK need.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fa {
+namespace bwd {
+
+constexpr int BM = 128;  // keys per CTA (MMA rows)
+constexpr int BQ = 128;  // queries per inner tile
+constexpr int D = 128;
+constexpr int TILE_BYTES = 128 * D * 2;
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int NUM_THREADS = 320;
+constexpr int MMA_WARP = 8;
+constexpr int TMA_WARP = 9;
+
+struct Smem {
+  uint8_t k[TILE_BYTES];
+  uint8_t v[TILE_BYTES];
+  uint8_t q[2][TILE_BYTES];
+  uint8_t dout[2][TILE_BYTES];
+  uint8_t ds[TILE_BYTES];  // dS as [query half][key][64 queries], 128-byte swizzle
+  float lse2[2][BQ];       // lse * log2(e) of the query tile (+inf past N)
+  float delta[2][BQ];
+  uint64_t kv_full;
+  uint64_t qdo_full[2];
+  uint64_t qdo_empty[2];
+  uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t kSmemBytes = sizeof(Smem);
+static_assert(kSmemBytes <= 232448, "backward shared memory exceeds the sm_100 limit");
+
+__device__ __forceinline__ void q_tile_range(int kt, int n, int causal, int window, int& lo, int& hi) {
+  const int k0 = kt * BM;
+  const int k1 = min(k0 + BM - 1, n - 1);
+  const int ntiles = (n + BQ - 1) / BQ;
+  lo = causal ? k0 / BQ : 0;
+  hi = ntiles;
+  if (window > 0) hi = min(hi, (k1 + window - 1) / BQ + 1);
+  if (lo > hi) lo = hi;
+}
+
+__device__ __forceinline__ bool tile_needs_mask(int kt, int qi, int n, int causal, int window) {
+  const int k0 = kt * BM, k1 = k0 + BM - 1;
+  const int q0 = qi * BQ, q1 = q0 + BQ - 1;
+  return (k1 >= n) || (causal && q0 < k1) || (window > 0 && q1 - k0 >= window);
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
+__device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(a_smem + off, 16, 1024), smem_desc_sw128(b_smem + off, 16, 1024),
+           idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// D[128 x d] (+)= A[tmem, 128 x 128 bf16] * B, B = [128 rows (K)][d] tile (MN-major).
+__device__ __forceinline__ void issue_tmemA_b(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
+                                              bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem).
+__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+#pragma unroll
+  for (int kk = 0; kk < BM / 16; ++kk)
+    mma_ss(d_tmem, smem_desc_sw128(ds_smem + kk * 2048, HALF_BYTES, 1024),
+           smem_desc_sw128(k_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    BwdArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusTimeout);
+    return;
+  }
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = args.N;
+  const int BH = args.B * args.H;
+  const int nkt = (n + BM - 1) / BM;
+  // Causal: low key tiles see the most query tiles -> launch them first.
+  const int kt = static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  (void)nkt;
+  int qlo, qhi;
+  q_tile_range(kt, n, args.causal, args.window, qlo, qhi);
+  const int nq = qhi - qlo;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&sm.kv_full), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&sm.qdo_full[s]), 1);
+      mbar_init(smem_u32(&sm.qdo_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&sm.s_full), 1);
+    mbar_init(smem_u32(&sm.dp_full), 1);
+    mbar_init(smem_u32(&sm.ds_ready), 128);
+    mbar_init(smem_u32(&sm.dq_full), 1);
+    mbar_init(smem_u32(&sm.dq_free), 128);
+    mbar_init(smem_u32(&sm.acc_done), 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  const uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 384;
+
+  if (warp == TMA_WARP) {
+    if (lane == 0 && nq > 0) {
+      const uint32_t kvb = smem_u32(&sm.kv_full);
+      mbar_arrive_expect_tx(kvb, 2 * TILE_BYTES);
+      tma_load_3d(smem_u32(sm.k), &tm_k, kvb, 0, kt * BM, bh);
+      tma_load_3d(smem_u32(sm.k) + HALF_BYTES, &tm_k, kvb, 64, kt * BM, bh);
+      tma_load_3d(smem_u32(sm.v), &tm_v, kvb, 0, kt * BM, bh);
+      tma_load_3d(smem_u32(sm.v) + HALF_BYTES, &tm_v, kvb, 64, kt * BM, bh);
+      int issued = 0;
+      for (int idx = 0; idx < nq; ++idx) {
+        const int s = idx & 1;
+        if (idx >= 2 && !mbar_wait(smem_u32(&sm.qdo_empty[s]), ((idx >> 1) - 1) & 1, abort_flag)) break;
+        const int row = (qlo + idx) * BQ;
+        const uint32_t b = smem_u32(&sm.qdo_full[s]);
+        mbar_arrive_expect_tx(b, 2 * TILE_BYTES);
+        tma_load_3d(smem_u32(sm.q[s]), &tm_q, b, 0, row, bh);
+        tma_load_3d(smem_u32(sm.q[s]) + HALF_BYTES, &tm_q, b, 64, row, bh);
+        tma_load_3d(smem_u32(sm.dout[s]), &tm_do, b, 0, row, bh);
+        tma_load_3d(smem_u32(sm.dout[s]) + HALF_BYTES, &tm_do, b, 64, row, bh);
+        issued = idx + 1;
+      }
+      mbar_wait_drain(kvb, 0);
+      for (int idx = max(0, issued - 2); idx < issued; ++idx)
+        mbar_wait_drain(smem_u32(&sm.qdo_full[idx & 1]), (idx >> 1) & 1);
+    }
+  } else if (warp == MMA_WARP) {
+    if (lane == 0 && nq > 0) {
+      const uint32_t ks = smem_u32(sm.k), vs = smem_u32(sm.v), dss = smem_u32(sm.ds);
+      bool ok = mbar_wait(smem_u32(&sm.kv_full), 0, abort_flag);
+      if (ok) ok = mbar_wait(smem_u32(&sm.qdo_full[0]), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_abT(tmem + T_S, ks, smem_u32(sm.q[0]));
+        tc_commit(smem_u32(&sm.s_full));
+        issue_abT(tmem + T_DP, vs, smem_u32(sm.dout[0]));
+        tc_commit(smem_u32(&sm.dp_full));
+      }
+      for (int idx = 0; ok && idx < nq; ++idx) {
+        const int s = idx & 1;
+        ok = mbar_wait(smem_u32(&sm.ds_ready), idx & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_tmemA_b(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
+        issue_tmemA_b(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
+        tc_commit(smem_u32(&sm.qdo_empty[s]));
+        issue_dq(tmem + T_S, dss, ks);
+        tc_commit(smem_u32(&sm.dq_full));
+        if (idx + 1 < nq) {
+          const int s1 = (idx + 1) & 1;
+          ok = mbar_wait(smem_u32(&sm.qdo_full[s1]), ((idx + 1) >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_abT(tmem + T_DP, vs, smem_u32(sm.dout[s1]));
+          tc_commit(smem_u32(&sm.dp_full));
+          ok = mbar_wait(smem_u32(&sm.dq_free), idx & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_abT(tmem + T_S, ks, smem_u32(sm.q[s1]));
+          tc_commit(smem_u32(&sm.s_full));
+        }
+      }
+      tc_commit(smem_u32(&sm.acc_done));
+      mbar_wait_drain(smem_u32(&sm.acc_done), 0);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // -------------------------------------------------- P^T and dS^T (thread = key row)
+    const int row = warp * 32 + lane;
+    const int key = kt * BM + row;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + T_S, tDP = tmem + lane_off + T_DP;
+    const float sl2 = args.scale_log2;
+    const float* lse_g = args.lse + static_cast<size_t>(bh) * n;
+    const float* del_g = args.ws_delta + static_cast<size_t>(bh) * n;
+    uint8_t* ds_row = sm.ds + row * 128;
+    bool ok = true;
+    // Prefetch the first tile's row statistics.
+    float lse_next = INFINITY, del_next = 0.f;
+    if (nq > 0) {
+      const int qi = qlo * BQ + row;
+      if (qi < n) {
+        const float l = lse_g[qi];
+        lse_next = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+        del_next = del_g[qi];
+      }
+    }
+    for (int idx = 0; idx < nq; ++idx) {
+      const int s = idx & 1;
+      sm.lse2[s][row] = lse_next;
+      sm.delta[s][row] = del_next;
+      named_bar_sync(1, 128);
+      if (idx + 1 < nq) {
+        const int qi = (qlo + idx + 1) * BQ + row;
+        lse_next = INFINITY;
+        del_next = 0.f;
+        if (qi < n) {
+          const float l = lse_g[qi];
+          lse_next = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+          del_next = del_g[qi];
+        }
+      }
+      const int qt = qlo + idx;
+      const bool masked = tile_needs_mask(kt, qt, n, args.causal, args.window);
+      ok = mbar_wait(smem_u32(&sm.s_full), idx & 1, abort_flag);
+      if (ok) ok = mbar_wait(smem_u32(&sm.dp_full), idx & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], dr[32];
+        FA_TMEM_LD32(tS + 32 * c, sr);
+        FA_TMEM_LD32(tDP + 32 * c, dr);
+        tmem_ld_wait();
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -sm.lse2[s][32 * c + e]));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), sl2, -sm.lse2[s][32 * c + e + 1]));
+          if (masked) {
+            const int q0 = qt * BQ + 32 * c + e;
+            if (!key_visible(q0, key, n, args.causal, args.window)) p0 = 0.f;
+            if (!key_visible(q0 + 1, key, n, args.causal, args.window)) p1 = 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(dr[e]) - sm.delta[s][32 * c + e]);
+          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - sm.delta[s][32 * c + e + 1]);
+          pp[e >> 1] = pack_bf16x2(p0, p1);
+          dd[e >> 1] = pack_bf16x2(d0, d1);
+        }
+        // P^T over S^T columns [16c, 16c+16), dS^T over dP^T columns (both already read).
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                tS + 16 * c),
+            "r"(pp[0]), "r"(pp[1]), "r"(pp[2]), "r"(pp[3]), "r"(pp[4]), "r"(pp[5]), "r"(pp[6]), "r"(pp[7]),
+            "r"(pp[8]), "r"(pp[9]), "r"(pp[10]), "r"(pp[11]), "r"(pp[12]), "r"(pp[13]), "r"(pp[14]),
+            "r"(pp[15])
+            : "memory");
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                tDP + 16 * c),
+            "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7]),
+            "r"(dd[8]), "r"(dd[9]), "r"(dd[10]), "r"(dd[11]), "r"(dd[12]), "r"(dd[13]), "r"(dd[14]),
+            "r"(dd[15])
+            : "memory");
+        // dS (queries 32c..32c+31 of this key row) into the swizzled MN-major tile.
+        uint8_t* half = ds_row + (c >> 1) * HALF_BYTES;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = ((c & 1) * 4 + u) ^ (row & 7);
+          *reinterpret_cast<uint4*>(half + chunk * 16) =
+              make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.ds_ready));
+    }
+    // Epilogue: dV rows.
+    if (ok && nq > 0) ok = mbar_wait(smem_u32(&sm.acc_done), 0, abort_flag);
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (nq > 0) {
+          FA_TMEM_LD32(tmem + lane_off + T_DV + 32 * c, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (key < n) {
+          uint4* o4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            o4[v4] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v4]), __uint_as_float(r[8 * v4 + 1])),
+                                pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3])),
+                                pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])),
+                                pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7])));
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------- dQ read-out (thread = query row)
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float scale = args.scale;
+    bool ok = true;
+    for (int idx = 0; idx < nq; ++idx) {
+      ok = mbar_wait(smem_u32(&sm.dq_full), idx & 1, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const int qi = (qlo + idx) * BQ + row;
+      float* acc = args.ws_dq + (static_cast<size_t>(bh) * n + qi) * D;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        FA_TMEM_LD32(tmem + lane_off + T_S + 32 * c, r);
+        tmem_ld_wait();
+        if (qi < n) {
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            red_add_v4(acc + 32 * c + 4 * v4, __uint_as_float(r[4 * v4]) * scale,
+                       __uint_as_float(r[4 * v4 + 1]) * scale, __uint_as_float(r[4 * v4 + 2]) * scale,
+                       __uint_as_float(r[4 * v4 + 3]) * scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.dq_free));
+    }
+    // Epilogue: dK rows (scaled).
+    if (ok && nq > 0) ok = mbar_wait(smem_u32(&sm.acc_done), 0, abort_flag);
+    const int key = kt * BM + row;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        if (nq > 0) {
+          FA_TMEM_LD32(tmem + lane_off + T_DK + 32 * c, r);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (key < n) {
+          uint4* o4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            o4[v4] = make_uint4(
+                pack_bf16x2(__uint_as_float(r[8 * v4]) * scale, __uint_as_float(r[8 * v4 + 1]) * scale),
+                pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * scale, __uint_as_float(r[8 * v4 + 3]) * scale),
+                pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * scale, __uint_as_float(r[8 * v4 + 5]) * scale),
+                pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * scale, __uint_as_float(r[8 * v4 + 7]) * scale));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D = rowsum(dO * O) in fp32 and a zeroed dQ accumulator; 16 lanes per row.
+__global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, long long rows) {
+  const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 4;
+  const int sub = threadIdx.x & 15;
+  float s = 0.f;
+  if (row < rows) {
+    const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o) + row * D + sub * 8);
+    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + row * D + sub * 8);
+    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      s = fmaf(__uint_as_float(ow[i] << 16), __uint_as_float(gw[i] << 16), s);
+      s = fmaf(__uint_as_float(ow[i] & 0xffff0000u), __uint_as_float(gw[i] & 0xffff0000u), s);
+    }
+    float4* acc = reinterpret_cast<float4*>(a.ws_dq + row * D + sub * 8);
+    acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (row < rows && sub == 0) a.ws_delta[row] = s;
+}
+
+// dQ accumulator (already scaled) -> bf16; 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_post_kernel(BwdArgs a, long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= n8) return;
+  const float4* src = reinterpret_cast<const float4*>(a.ws_dq) + 2 * i;
+  const float4 x = src[0], y = src[1];
+  reinterpret_cast<uint4*>(a.dq)[i] =
+      make_uint4(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w), pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+}
+
+}  // namespace bwd
+
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  using namespace bwd;
+  const long long bh = static_cast<long long>(a.B) * a.H;
+  const long long rows = bh * a.N;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap_bf16_rows(&tq, a.q, D, a.N, bh, BQ) || !make_tmap_bf16_rows(&tk, a.k, D, a.N, bh, BM) ||
+      !make_tmap_bf16_rows(&tv, a.v, D, a.N, bh, BM) || !make_tmap_bf16_rows(&tdo, a.dout, D, a.N, bh, BQ))
+    return cudaErrorInvalidValue;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(bwd_main_kernel), kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const long long pre_blocks = (rows * 16 + 255) / 256;
+  if (pre_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  bwd_pre_kernel<<<static_cast<unsigned>(pre_blocks), 256, 0, stream>>>(a, rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long nkt = (a.N + BM - 1) / BM;
+  bwd_main_kernel<<<static_cast<unsigned>(nkt * bh), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n8 = rows * D / 8;
+  bwd_post_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(a, n8);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,182 @@
+// Single-token decode against a padded key/value cache (bf16, d = 128).
+//
+// "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
+// Python", Step 4: the query of (b, h) attends to every cached position
+// j < seqlens[b] (the cache already holds the current token).  The work is
+// HBM-bound: every cached key and value row is read once, 256 bytes each.
+//
+// Split: CTA (chunk, h, b) scores keys [chunk * 512, chunk * 512 + 512) of
+// its sequence with the online softmax and writes a normalised partial
+// (o_c, lse_c).  Each half-warp owns one key row per step (16 lanes x 16
+// bytes = one 256-byte row, so a warp reads 512 contiguous bytes per load
+// instruction) and keeps 8 rows of K and 8 of V in flight per thread.
+// Combine: lse = ln sum_c exp(lse_c), o = sum_c exp(lse_c - lse) o_c -- the
+// two-softmax merge identity of "Building Flash Attention from Scratch in
+// Pure NumPy" (architecture overview), restated.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fa {
+namespace dec {
+
+constexpr int D = 128;
+constexpr int THREADS = 256;          // 8 warps = 16 half-warps
+constexpr int HALVES = THREADS / 16;
+constexpr int U = 8;                  // key rows in flight per half-warp and step
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__global__ void __launch_bounds__(THREADS)
+    decode_split_kernel(DecodeArgs a) {
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n = min(max(a.seqlens[b], 0), a.cap);
+  const int start = c * kDecodeChunk;
+  if (start >= n) return;
+  const int end = min(start + kDecodeChunk, n);
+
+  const int lane = threadIdx.x & 31;
+  const int hw = threadIdx.x >> 4;   // half-warp 0..15
+  const int sub = lane & 15;         // 16-byte slice of the row
+  const size_t bhh = static_cast<size_t>(b) * a.H + h;
+
+  float qf[8];
+  bf16x8_to_f32(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + bhh * D + sub * 8), qf);
+  const float sl2 = a.scale_log2;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) qf[e] *= sl2;  // scores come out in exp2 units
+
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.kcache) + bhh * a.cap * D + sub * 8;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(a.vcache) + bhh * a.cap * D + sub * 8;
+
+  float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+
+  for (int key0 = start + hw; key0 < end; key0 += HALVES * U) {
+    uint4 kr[U], vr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int key = key0 + u * HALVES;
+      if (key < end) {
+        kr[u] = ld_stream(kb + static_cast<size_t>(key) * D);
+        vr[u] = ld_stream(vb + static_cast<size_t>(key) * D);
+      } else {
+        kr[u] = make_uint4(0, 0, 0, 0);
+        vr[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    float s[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float kf[8];
+      bf16x8_to_f32(kr[u], kf);
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      s[u] = (key0 + u * HALVES < end) ? dot : -INFINITY;
+    }
+    float mx = s[0];
+#pragma unroll
+    for (int u = 1; u < U; ++u) mx = fmaxf(mx, s[u]);
+    const float m_new = fmaxf(m, mx);  // finite: key0 < end makes s[0] finite
+    const float alpha = ex2_approx(m - m_new);
+    l *= alpha;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] *= alpha;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float p = ex2_approx(s[u] - m_new);
+      l += p;
+      float vf[8];
+      bf16x8_to_f32(vr[u], vf);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
+    }
+    m = m_new;
+  }
+
+  // Merge the 16 half-warp states (exp2 units) through shared memory.
+  __shared__ float sm_m[HALVES], sm_l[HALVES];
+  __shared__ float sm_acc[HALVES][D];
+  if (sub == 0) {
+    sm_m[hw] = m;
+    sm_l[hw] = l;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sm_acc[hw][sub * 8 + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int e = threadIdx.x;
+    float M = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < HALVES; ++i) M = fmaxf(M, sm_m[i]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int i = 0; i < HALVES; ++i) {
+      const float w = (sm_m[i] == -INFINITY) ? 0.f : ex2_approx(sm_m[i] - M);
+      L = fmaf(sm_l[i], w, L);
+      O = fmaf(sm_acc[i][e], w, O);
+    }
+    const size_t row = bhh * a.max_chunks + c;
+    a.ws_o[row * D + e] = O / L;
+    if (e == 0) a.ws_lse[row] = (M + log2f(L)) * 0.69314718055994531f;  // natural log
+  }
+}
+
+__global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
+  const size_t bhh = blockIdx.x;
+  const int b = static_cast<int>(bhh / a.H);
+  const int n = min(max(a.seqlens[b], 0), a.cap);
+  const int chunks = (n + kDecodeChunk - 1) / kDecodeChunk;
+  const int e = threadIdx.x;
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o) + bhh * D;
+  if (chunks == 0) {
+    o[e] = __float2bfloat16_rn(0.f);
+    if (e == 0 && a.lse) a.lse[bhh] = -INFINITY;
+    return;
+  }
+  const float* ls = a.ws_lse + bhh * a.max_chunks;
+  const float* os = a.ws_o + bhh * a.max_chunks * D;
+  float M = -INFINITY;
+  for (int c = 0; c < chunks; ++c) M = fmaxf(M, ls[c]);
+  float W = 0.f, O = 0.f;
+  for (int c = 0; c < chunks; ++c) {
+    const float w = __expf(ls[c] - M);
+    W += w;
+    O = fmaf(w, os[static_cast<size_t>(c) * D + e], O);
+  }
+  o[e] = __float2bfloat16_rn(O / W);
+  if (e == 0 && a.lse) a.lse[bhh] = M + logf(W);
+}
+
+}  // namespace dec
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  using namespace dec;
+  if (a.H > 65535 || a.B > 65535) return cudaErrorInvalidValue;
+  dim3 grid(a.max_chunks, a.H, a.B);
+  decode_split_kernel<<<grid, THREADS, 0, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<<<static_cast<unsigned>(a.B * a.H), D, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

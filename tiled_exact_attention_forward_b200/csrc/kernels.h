@@ -1,0 +1,71 @@
+// Internal launch interface between the C ABI (fa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fa {
+
+struct FwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;  // may be null
+  int B, H, N, d;
+  int causal, window;
+  float scale;       // natural units
+  float scale_log2;  // scale * log2(e)
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* kcache;
+  const void* vcache;
+  const int32_t* seqlens;
+  void* o;
+  float* lse;  // may be null
+  int B, H, cap, d;
+  float scale, scale_log2;
+  float* ws_o;    // [B*H][max_chunks][d] normalised chunk outputs
+  float* ws_lse;  // [B*H][max_chunks] chunk logsumexp
+  int max_chunks;
+};
+
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  int B, H, N, d;
+  int causal, window;
+  float scale, scale_log2;
+  float* ws_delta;  // [B*H*N] rowsum(dO * O)
+  float* ws_dq;     // [B*H*N*d] fp32 dQ accumulator
+};
+
+// Decode: keys per split chunk (one CTA each).
+constexpr int kDecodeChunk = 512;
+
+inline int decode_max_chunks(int cap) { return (cap + kDecodeChunk - 1) / kDecodeChunk; }
+
+// Host helpers (fa_host.cu).
+// A 3-D TMA map over a bf16 [heads][rows_per_head][d] array: boxes of 64
+// columns x box_rows rows, 128-byte swizzle, rows past the end read as zero.
+bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_head,
+                         long long heads, int box_rows);
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device and kernel.
+cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+
+}  // namespace fa
