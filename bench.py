@@ -277,6 +277,20 @@ def make_step(w, dev):
             ["bwd.cu" if with_bwd else "fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank values (the slowest rank sets the time)."""
+    import torch.distributed as tdist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms: float) -> float:
+    """Work of all ranks (weak scaling: each rank its own batch) per second."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def timed_loop(fn, steps, warmup, flush, stream):
     for _ in range(warmup):
         fn()
@@ -324,11 +338,9 @@ def run_gpu(args, rank, world, local_rank):
     barrier()
     e2e_ms = float(np.mean(e2e_times))
     if dist:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-    value = units * world / (ms / 1e3)
-    e2e_value = units * world / (e2e_ms / 1e3)
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], device=dev)
+    value = whole_job_rate(units, world, ms)
+    e2e_value = whole_job_rate(units, world, e2e_ms)
     hbm, tflops, peak_kind = load_peaks()
     if unit == "GB/s":
         roof = {"bound": "hbm", "achieved": units / (ms / 1e3), "peak": hbm, "unit": "GB/s"}

@@ -153,6 +153,16 @@ FA_API fa_status fa_backward(const void* q, const void* k, const void* v, const 
  */
 FA_API fa_status fa_get_device_status(void* stream);
 
+/*
+ * Failure-path self-test: launches one CTA whose only thread block waits on
+ * an internal barrier that nothing ever completes, with a bound of
+ * `limit_cycles` SM clock cycles (1 .. 4e9).  The wait gives up, the kernel
+ * records FA_ERR_TIMEOUT and returns normally, exactly as every production
+ * kernel does when a barrier stalls; the next fa_get_device_status() on
+ * `stream` reports it and clears it.  The CUDA context stays usable.
+ */
+FA_API fa_status fa_selftest_wait_timeout(long long limit_cycles, void* stream);
+
 /* Static, human-readable name of a status code. */
 FA_API const char* fa_status_string(fa_status status);
 

@@ -3,7 +3,10 @@
 Tolerances (fixed by the task's stated bar, written here once):
   forward / decode outputs: max |err| <= 2e-2 and mean |err| <= 2e-3
   logsumexp:                max |err| <= 1e-3
-  gradients:                max |err| <= 5e-2 * max |reference gradient|
+  gradients:                max |err| <= 5e-2 * max |reference gradient|, with an
+                            absolute floor of 1e-4 for gradients that vanish
+                            identically (one visible key per query makes dS = 0,
+                            so dQ = dK = 0 and a purely relative bound is empty)
   float32 forward:          max |err| <= 1e-4 (the NumPy page's allclose atol)
 """
 import numpy as np
@@ -14,6 +17,7 @@ OUT_MAX = 2e-2
 OUT_MEAN = 2e-3
 LSE_MAX = 1e-3
 GRAD_REL = 5e-2
+GRAD_FLOOR = 1e-4
 FP32_ATOL = 1e-4
 
 requires_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
@@ -37,14 +41,15 @@ def assert_output_close(got, ref, what, max_tol=OUT_MAX, mean_tol=OUT_MEAN):
 def assert_lse_close(got, ref, what, tol=LSE_MAX):
     got, ref = to64(got), to64(ref)
     both_inf = np.isneginf(got) & np.isneginf(ref)
-    err = np.abs(np.where(both_inf, 0.0, got - ref))
+    with np.errstate(invalid="ignore"):
+        err = np.abs(np.where(both_inf, 0.0, got - ref))
     assert np.all(np.isfinite(err)), f"{what}: lse mismatch in -inf pattern"
     assert err.max() <= tol, f"{what}: lse max |err| {err.max():.3g} > {tol}"
 
 
-def assert_grad_close(got, ref, what, rel=GRAD_REL):
+def assert_grad_close(got, ref, what, rel=GRAD_REL, floor=GRAD_FLOOR):
     got, ref = to64(got), to64(ref)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
-    scale = max(np.abs(ref).max(), 1e-30)
+    tol = max(rel * np.abs(ref).max(), floor)
     err = np.abs(got - ref).max()
-    assert err <= rel * scale, f"{what}: max |err| {err:.3g} > {rel} * {scale:.3g}"
+    assert err <= tol, f"{what}: max |err| {err:.3g} > {tol:.3g}"

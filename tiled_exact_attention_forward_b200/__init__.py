@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = (
     "fa_backward_workspace_size",
     "fa_backward",
     "fa_get_device_status",
+    "fa_selftest_wait_timeout",
     "fa_status_string",
     "fa_version",
 )
@@ -71,6 +72,8 @@ def _lib() -> ctypes.CDLL:
     lib.fa_backward_workspace_size.restype = Z
     lib.fa_backward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, I, I, P, Z, P]
     lib.fa_backward.restype = I
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
+    lib.fa_selftest_wait_timeout.restype = I
     lib.fa_get_device_status.argtypes = [P]
     lib.fa_get_device_status.restype = I
     lib.fa_status_string.argtypes = [I]
@@ -213,6 +216,12 @@ def backward(q, k, v, o, dout, lse, causal: bool = False, window: int = 0, scale
                             _stream(q.device))
     _check(st, "fa_backward")
     return dq, dk, dv
+
+
+def selftest_wait_timeout(limit_cycles: int = 20_000_000, device=None) -> int:
+    """Run the failure-path self-test kernel (a bounded wait that must expire)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(_lib().fa_selftest_wait_timeout(int(limit_cycles), _stream(dev)))
 
 
 def device_status(device=None) -> int:

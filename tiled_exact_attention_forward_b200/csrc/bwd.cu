@@ -79,7 +79,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
+__device__ __forceinline__ void named_bar_sync(int id, int count) {  // bar.sync id, count
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
@@ -266,6 +266,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool masked = tile_needs_mask(kt, qt, n, args.causal, args.window);
       ok = mbar_wait(smem_u32(&sm.s_full), idx & 1, abort_flag);
       if (ok) ok = mbar_wait(smem_u32(&sm.dp_full), idx & 1, abort_flag);
+      // One decision for the whole warpgroup: it meets at named barrier 1 every step.
+      ok = named_bar_all(ok, 2, 128);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
@@ -319,7 +321,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(smem_u32(&sm.ds_ready));
     }
     // Epilogue: dV rows.
-    if (ok && nq > 0) ok = mbar_wait(smem_u32(&sm.acc_done), 0, abort_flag);
+    if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D;
     if (ok) {
       tc_fence_after();
@@ -352,7 +354,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float scale = args.scale;
     bool ok = true;
     for (int idx = 0; idx < nq; ++idx) {
-      ok = mbar_wait(smem_u32(&sm.dq_full), idx & 1, abort_flag);
+      ok = mbar_wait_warp(smem_u32(&sm.dq_full), idx & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const int qi = (qlo + idx) * BQ + row;
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_arrive(smem_u32(&sm.dq_free));
     }
     // Epilogue: dK rows (scaled).
-    if (ok && nq > 0) ok = mbar_wait(smem_u32(&sm.acc_done), 0, abort_flag);
+    if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
     const int key = kt * BM + row;
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D;
     if (ok) {

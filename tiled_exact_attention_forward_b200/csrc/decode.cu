@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(THREADS)
   const int end = min(start + kDecodeChunk, n);
 
   const int lane = threadIdx.x & 31;
-  const int hw = threadIdx.x >> 4;   // half-warp 0..15
+  const int hw = threadIdx.x >> 4;   // half-warp 0..15 (keys start + hw + 16 i)
   const int sub = lane & 15;         // 16-byte slice of the row
   const size_t bhh = static_cast<size_t>(b) * a.H + h;
 
@@ -67,11 +67,15 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 
-  for (int key0 = start + hw; key0 < end; key0 += HALVES * U) {
+  // The loop bound is warp-uniform (both half-warps run the same trip count), so the
+  // full-warp shuffles below always see all 32 lanes; each key is checked on its own.
+  const int half = (threadIdx.x >> 4) & 1;
+  const int warp = threadIdx.x >> 5;
+  for (int kbase = start + 2 * warp; kbase < end; kbase += HALVES * U) {
     uint4 kr[U], vr[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int key = key0 + u * HALVES;
+      const int key = kbase + half + u * HALVES;
       if (key < end) {
         kr[u] = ld_stream(kb + static_cast<size_t>(key) * D);
         vr[u] = ld_stream(vb + static_cast<size_t>(key) * D);
@@ -90,19 +94,22 @@ __global__ void __launch_bounds__(THREADS)
       for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      s[u] = (key0 + u * HALVES < end) ? dot : -INFINITY;
+      s[u] = (kbase + half + u * HALVES < end) ? dot : -INFINITY;
     }
     float mx = s[0];
 #pragma unroll
     for (int u = 1; u < U; ++u) mx = fmaxf(mx, s[u]);
-    const float m_new = fmaxf(m, mx);  // finite: key0 < end makes s[0] finite
-    const float alpha = ex2_approx(m - m_new);
+    const float m_new = fmaxf(m, mx);
+    // A half-warp may have no valid key in this step (and none before): keep its
+    // state unchanged instead of forming (-inf) - (-inf).
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+    const float alpha = ex2_approx(m - m_use);  // m = -inf gives 0: nothing accumulated yet
     l *= alpha;
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] *= alpha;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const float p = ex2_approx(s[u] - m_new);
+      const float p = ex2_approx(s[u] - m_use);
       l += p;
       float vf[8];
       bf16x8_to_f32(vr[u], vf);

@@ -131,6 +131,11 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   return from_cuda(fa::launch_bwd(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1 || limit_cycles > 4000000000LL) return FA_ERR_INVALID;
+  return from_cuda(fa::launch_selftest_wait_timeout(limit_cycles, static_cast<cudaStream_t>(stream)));
+}
+
 fa_status fa_get_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);

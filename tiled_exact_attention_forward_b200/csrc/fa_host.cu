@@ -67,4 +67,30 @@ cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   return cudaSuccess;
 }
 
+namespace {
+
+// One CTA waits on an mbarrier that nothing ever arrives on.  The bounded wait
+// must give up after `limit_cycles`, record the timeout in the status word and
+// let the kernel return normally -- the same path every production kernel
+// takes when a barrier stalls.
+__global__ void selftest_wait_timeout_kernel(long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, limit_cycles);
+  (void)ok;
+}
+
+}  // namespace
+
+cudaError_t launch_selftest_wait_timeout(long long limit_cycles, cudaStream_t stream) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_cycles);
+  return cudaGetLastError();
+}
+
 }  // namespace fa

@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int it = 0;
     if (t == 0 || has1) {
       for (int j = lo_t[t]; j < hi_t[t]; ++j, ++it) {
-        ok = mbar_wait(smem_u32(&sm.s_full[t]), it & 1, abort_flag);
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), it & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         uint32_t s[BN];
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         l += rs;
       }
       // Epilogue: O / l in bf16 and lse = m * scale + ln l.
-      if (ok && hi_t[t] > lo_t[t]) ok = mbar_wait(smem_u32(&sm.o_full[t]), 0, abort_flag);
+      if (ok && hi_t[t] > lo_t[t]) ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
