@@ -120,6 +120,30 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this exists for deployment, not for the method.  Same arguments,
+ * layout and results as fa_decode, minus the workspace: the per-chunk
+ * partials go to a fixed array of FA_DECODE_NOALLOC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  Serving runtimes that forbid allocation after start-up and plugin
+ * interfaces that pass a kernel only its inputs and outputs are the intended
+ * users.
+ *   - Size limit: fa_decode_workspace_size(B, H, cap, d) must not exceed
+ *     FA_DECODE_NOALLOC_SCRATCH_BYTES (for cap = 8192 that is B*H <= 1016);
+ *     larger calls return FA_ERR_INVALID with nothing launched.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls share the array: calls whose kernels overlap on the GPU race.
+ *     Nothing needs clearing between calls.
+ *   - Calls no cudaMalloc/cudaFree and no allocating library routine.
+ */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+FA_API fa_status fa_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                   const int32_t* seqlens, void* o, float* lse,
+                                   int B, int H, int cap, int d, float scale, fa_dtype dtype,
+                                   void* stream);
+
+/*
  * Bytes of device workspace fa_backward needs (a multiple of 256): the
  * float32 row terms D = rowsum(dO * O) and a float32 dQ accumulator.
  */

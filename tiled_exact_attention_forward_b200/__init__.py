@@ -31,6 +31,7 @@ EXPORTED_SYMBOLS = (
     "fa_forward",
     "fa_decode_workspace_size",
     "fa_decode",
+    "fa_decode_noalloc",
     "fa_backward_workspace_size",
     "fa_backward",
     "fa_get_device_status",
@@ -68,6 +69,8 @@ def _lib() -> ctypes.CDLL:
     lib.fa_decode_workspace_size.restype = Z
     lib.fa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
     lib.fa_decode.restype = I
+    lib.fa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P]
+    lib.fa_decode_noalloc.restype = I
     lib.fa_backward_workspace_size.argtypes = [I, I, I, I]
     lib.fa_backward_workspace_size.restype = Z
     lib.fa_backward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, I, I, P, Z, P]
