@@ -312,7 +312,7 @@ def run_gpu(args, rank, world, local_rank):
     import tiled_exact_attention_forward_b200 as fa
 
     fa.library()
-    w = workloads.WORKLOADS[args.workload]
+    w = resolve_workload(args)
     (step, e2e, units, unit, metric, launches, kernel, sources, h2d, d2h) = make_step(w, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -370,8 +370,17 @@ def run_gpu(args, rank, world, local_rank):
     return line
 
 
-def run_reference(args):
+def resolve_workload(args):
+    """The named workload, with the batch/head overrides used for small profiling runs."""
+    import dataclasses
+
     w = workloads.WORKLOADS[args.workload]
+    changes = {k: v for k, v in (("B", args.B), ("H", args.H)) if v is not None}
+    return dataclasses.replace(w, **changes) if changes else w
+
+
+def run_reference(args):
+    w = resolve_workload(args)
     t0 = time.perf_counter()
     vals = []
     samples = []
@@ -406,6 +415,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=4.0)
+    ap.add_argument("--B", type=int, default=None, help="override the workload's batch (profiling)")
+    ap.add_argument("--H", type=int, default=None, help="override the workload's heads (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -256,6 +256,74 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ---------------------------------------------------------------- packed fp32 (sm_100 f32x2)
+// Two floats in one 64-bit register pair; fma/add/sub/mul.rn.f32x2 process both
+// in one instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max of three floats that is NaN when any input is NaN.
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (no special-function unit):
+// x = j + f with j = round(x) (the 1.5 * 2^23 rounding trick) and
+// f in [-0.5, 0.5]; 2^f from a cubic fitted for minimum relative error on that
+// interval (max 7.5e-5; derivation in fit_exp2_poly.py); 2^j added to the
+// exponent field.  x is clamped to >= -126.5 so 2^j stays a normal scale: for
+// x below that the result is a tiny positive number (< 1e-38) instead of 0,
+// far under bf16's resolution of P.  A NaN input does NOT come out as NaN
+// (the clamp drops it); callers that must propagate NaN check for it apart.
+__device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -126.5f), fmaxf(x1, -126.5f));
+  const uint64_t kMagic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x2, kMagic);       // integer part in the low mantissa bits
+  const uint64_t j = f2_sub(t, kMagic);        // round(x)
+  const uint64_t f = f2_sub(x2, j);            // in [-0.5, 0.5]
+  uint64_t p = f2_fma(f2_pack(0.055171623826026917f, 0.055171623826026917f), f,
+                      f2_pack(0.24261116981506348f, 0.24261116981506348f));
+  p = f2_fma(p, f, f2_pack(0.6932610273361206f, 0.6932610273361206f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // bits(t) = bits(1.5 * 2^23) + j; shifting left by 23 leaves exactly j << 23.
+  const uint32_t r0 = (__float_as_uint(t0) << 23) + __float_as_uint(p0);
+  const uint32_t r1 = (__float_as_uint(t1) << 23) + __float_as_uint(p1);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -67,6 +67,24 @@ cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   return cudaSuccess;
 }
 
+cudaError_t sm_count(int* out) {
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    cached[dev] = v;
+  }
+  *out = cached[dev];
+  return cudaSuccess;
+}
+
 namespace {
 
 // One CTA waits on an mbarrier that nothing ever arrives on.  The bounded wait

@@ -56,11 +56,13 @@ struct Smem {
   uint8_t q[2][TILE_BYTES];
   uint8_t kv[NS][TILE_BYTES];
   uint64_t q_full[2];
+  uint64_t q_empty[2];
   uint64_t kv_full[NS];
   uint64_t kv_empty[NS];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
+  uint64_t o_free[2];
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -107,6 +109,46 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   }
 }
 
+// One unit of work: two 128-row query tiles (rows [256p, 256p + 256)) of one
+// (batch, head), with the key-tile range each of them must visit.
+struct Item {
+  int bh;
+  int r0[2];
+  int lo_t[2], hi_t[2];
+  int lo, hi;
+  bool has1;
+};
+
+__device__ __forceinline__ Item make_item(int lin, int BH, int n, int num_pairs, int causal, int window) {
+  Item it;
+  // Heaviest work first: with a causal mask the last query tiles see the most keys.
+  const int pair = num_pairs - 1 - lin / BH;
+  it.bh = lin % BH;
+  it.r0[0] = pair * 2 * BM;
+  it.r0[1] = it.r0[0] + BM;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (it.r0[t] < n) {
+      key_tile_range(it.r0[t], n, causal, window, it.lo_t[t], it.hi_t[t]);
+    } else {
+      it.lo_t[t] = it.hi_t[t] = 0;
+    }
+  }
+  it.has1 = it.r0[1] < n;
+  it.lo = it.has1 ? min(it.lo_t[0], it.lo_t[1]) : it.lo_t[0];
+  it.hi = it.has1 ? max(it.hi_t[0], it.hi_t[1]) : it.hi_t[0];
+  return it;
+}
+
+// Item index of round k for this CTA: items are sorted heaviest first and
+// dealt in a snake order (0..G-1, then G-1..0, ...) so every CTA gets a
+// similar total.  Returns -1 past the end.
+__device__ __forceinline__ int item_of(int k, int total) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const int lin = k * G + ((k & 1) ? (G - 1 - c) : c);
+  return lin < total ? lin : -1;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, FwdArgs args) {
@@ -118,31 +160,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int BH = args.B * args.H;
   const int n = args.N;
   const int num_pairs = (n + 2 * BM - 1) / (2 * BM);
-  // Heaviest work first: with a causal mask the last query tiles see the most keys.
-  const int pair = num_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-
-  int r0[2], lo_t[2], hi_t[2];
-  r0[0] = pair * 2 * BM;
-  r0[1] = r0[0] + BM;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    if (r0[t] < n) {
-      key_tile_range(r0[t], n, args.causal, args.window, lo_t[t], hi_t[t]);
-    } else {
-      lo_t[t] = hi_t[t] = 0;
-    }
-  }
-  const bool has1 = r0[1] < n;
-  const int lo = has1 ? min(lo_t[0], lo_t[1]) : lo_t[0];
-  const int hi = has1 ? max(hi_t[0], hi_t[1]) : hi_t[0];
+  const int total = num_pairs * BH;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(smem_u32(&sm.q_full[t]), 1);
+      mbar_init(smem_u32(&sm.q_empty[t]), 1);
       mbar_init(smem_u32(&sm.s_full[t]), 1);
       mbar_init(smem_u32(&sm.p_full[t]), BM);
       mbar_init(smem_u32(&sm.o_full[t]), 1);
+      mbar_init(smem_u32(&sm.o_free[t]), BM);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), 1);
@@ -170,32 +197,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == TMA_WARP) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int nt = has1 ? 2 : 1;
-      for (int t = 0; t < nt; ++t) {
-        const uint32_t bar = smem_u32(&sm.q_full[t]);
-        mbar_arrive_expect_tx(bar, TILE_BYTES);
-        tma_load_3d(smem_u32(sm.q[t]), &tm_q, bar, 0, r0[t], bh);
-        tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, r0[t], bh);
-      }
-      const int total = 2 * (hi - lo);
-      int issued = 0;
-      for (int idx = 0; idx < total; ++idx) {
-        const int s = idx % NS;
-        if (idx >= NS) {
-          if (!mbar_wait(smem_u32(&sm.kv_empty[s]), ((idx / NS) - 1) & 1, abort_flag)) break;
+      int nq[2] = {0, 0};  // Q tiles loaded so far, per slot
+      int kvi = 0;         // K/V ring fills so far (K and V interleaved)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int lin = item_of(k, total);
+        if (lin < 0) break;
+        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+        for (int t = 0; t < (it.has1 ? 2 : 1) && ok; ++t) {
+          // The slot is free once the previous item's last S_t MMA has completed.
+          if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
+          if (!ok) break;
+          const uint32_t bar = smem_u32(&sm.q_full[t]);
+          mbar_arrive_expect_tx(bar, TILE_BYTES);
+          tma_load_3d(smem_u32(sm.q[t]), &tm_q, bar, 0, it.r0[t], it.bh);
+          tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, it.r0[t], it.bh);
+          ++nq[t];
         }
-        const int j = lo + (idx >> 1);
-        const CUtensorMap* tm = (idx & 1) ? &tm_v : &tm_k;
-        const uint32_t bar = smem_u32(&sm.kv_full[s]);
-        mbar_arrive_expect_tx(bar, TILE_BYTES);
-        tma_load_3d(smem_u32(sm.kv[s]), tm, bar, 0, j * BN, bh);
-        tma_load_3d(smem_u32(sm.kv[s]) + HALF_BYTES, tm, bar, 64, j * BN, bh);
-        issued = idx + 1;
+        for (int idx = 0; ok && idx < 2 * (it.hi - it.lo); ++idx, ++kvi) {
+          const int s = kvi % NS;
+          if (kvi >= NS) ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((kvi / NS) - 1) & 1, abort_flag);
+          if (!ok) break;
+          const int j = it.lo + (idx >> 1);
+          const CUtensorMap* tm = (idx & 1) ? &tm_v : &tm_k;
+          const uint32_t bar = smem_u32(&sm.kv_full[s]);
+          mbar_arrive_expect_tx(bar, TILE_BYTES);
+          tma_load_3d(smem_u32(sm.kv[s]), tm, bar, 0, j * BN, it.bh);
+          tma_load_3d(smem_u32(sm.kv[s]) + HALF_BYTES, tm, bar, 64, j * BN, it.bh);
+        }
       }
       // Drain: every copy issued must land before the CTA may exit.
-      for (int idx = max(0, issued - NS); idx < issued; ++idx)
-        mbar_wait_drain(smem_u32(&sm.kv_full[idx % NS]), (idx / NS) & 1);
-      for (int t = 0; t < nt; ++t) mbar_wait_drain(smem_u32(&sm.q_full[t]), 0);
+      for (int i = max(0, kvi - NS); i < kvi; ++i) mbar_wait_drain(smem_u32(&sm.kv_full[i % NS]), (i / NS) & 1);
+      for (int t = 0; t < 2; ++t)
+        if (nq[t] > 0) mbar_wait_drain(smem_u32(&sm.q_full[t]), (nq[t] - 1) & 1);
     }
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -203,73 +237,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tS[2] = {tmem + 0, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
       const uint32_t q_s[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-      int it[2] = {0, 0};
+      int nq[2] = {0, 0};    // Q tiles consumed, per slot
+      int npv[2] = {0, 0};   // PV MMAs issued, per tile slot (p_full phase)
+      int nout[2] = {0, 0};  // items finished, per tile slot (o_free phase)
+      int kvi = 0;
       bool ok = true;
-      auto act = [&](int t, int j) { return j >= lo_t[t] && j < hi_t[t]; };
-      auto stage_of = [&](int idx) { return idx % NS; };
-      auto parity_of = [&](int idx) { return static_cast<uint32_t>((idx / NS) & 1); };
-
-      ok = mbar_wait(smem_u32(&sm.q_full[0]), 0, abort_flag);
-      if (ok && has1) ok = mbar_wait(smem_u32(&sm.q_full[1]), 0, abort_flag);
-      if (ok && hi > lo) {
-        // Prologue: S_t(lo) for both tiles.
-        int kidx = 0;
-        ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kidx)]), parity_of(kidx), abort_flag);
-        if (ok) {
+      auto stage_of = [&](int i) { return i % NS; };
+      auto parity_of = [&](int i) { return static_cast<uint32_t>((i / NS) & 1); };
+      for (int k = 0; ok; ++k) {
+        const int lin = item_of(k, total);
+        if (lin < 0) break;
+        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+        auto act = [&](int t, int j) { return j >= it.lo_t[t] && j < it.hi_t[t]; };
+        // S_t(j) and its bookkeeping: the last S_t of the item frees the Q slot.
+        auto issue_s = [&](int t, int j, uint32_t ks) {
+          issue_qk(tS[t], q_s[t], ks);
+          tc_commit(smem_u32(&sm.s_full[t]));
+          if (j == it.hi_t[t] - 1) tc_commit(smem_u32(&sm.q_empty[t]));
+        };
+        // PV_t(j): the first one of an item overwrites O_t, so the previous item's
+        // epilogue must have read it out; the last one publishes O_t.
+        auto issue_o = [&](int t, int j, uint32_t vs) -> bool {
+          if (j == it.lo_t[t] && nout[t] > 0) {
+            if (!mbar_wait(smem_u32(&sm.o_free[t]), (nout[t] - 1) & 1, abort_flag)) return false;
+          }
+          if (!mbar_wait(smem_u32(&sm.p_full[t]), npv[t] & 1, abort_flag)) return false;
           tc_fence_after();
-          const uint32_t ks = smem_u32(sm.kv[stage_of(kidx)]);
-          for (int t = 0; t < 2; ++t)
-            if (act(t, lo)) {
-              issue_qk(tS[t], q_s[t], ks);
-              tc_commit(smem_u32(&sm.s_full[t]));
-            }
-          tc_commit(smem_u32(&sm.kv_empty[stage_of(kidx)]));
+          issue_pv(tO[t], tS[t], vs, j > it.lo_t[t]);
+          ++npv[t];
+          if (j == it.hi_t[t] - 1) {
+            tc_commit(smem_u32(&sm.o_full[t]));
+            ++nout[t];
+          }
+          return true;
+        };
+        for (int t = 0; t < (it.has1 ? 2 : 1) && ok; ++t) {
+          ok = mbar_wait(smem_u32(&sm.q_full[t]), nq[t] & 1, abort_flag);
+          ++nq[t];
         }
-        for (int j = lo; ok && j < hi; ++j) {
-          const int vidx = 2 * (j - lo) + 1;
-          const int nidx = vidx + 1;
-          const bool has_next = j + 1 < hi;
+        if (!ok || it.hi <= it.lo) break;
+        // Prologue: S_t(lo) for both tiles.
+        ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi)]), parity_of(kvi), abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          const uint32_t ks = smem_u32(sm.kv[stage_of(kvi)]);
+          for (int t = 0; t < 2; ++t)
+            if (act(t, it.lo)) issue_s(t, it.lo, ks);
+          tc_commit(smem_u32(&sm.kv_empty[stage_of(kvi)]));
+          ++kvi;
+        }
+        for (int j = it.lo; ok && j < it.hi; ++j) {
+          const int vidx = kvi;            // V_j
+          const int nidx = kvi + 1;        // K_{j+1}
+          const bool has_next = j + 1 < it.hi;
           ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(vidx)]), parity_of(vidx), abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t vs = smem_u32(sm.kv[stage_of(vidx)]);
-          // Tile 0: PV0(j), then S0(j+1).
-          if (act(0, j)) {
-            ok = mbar_wait(smem_u32(&sm.p_full[0]), it[0] & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(tO[0], tS[0], vs, it[0] > 0);
-            ++it[0];
-            if (j == hi_t[0] - 1) tc_commit(smem_u32(&sm.o_full[0]));
-          }
+          if (act(0, j) && !(ok = issue_o(0, j, vs))) break;
           uint32_t ks = 0;
           if (has_next) {
             ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(nidx)]), parity_of(nidx), abort_flag);
             if (!ok) break;
             tc_fence_after();
             ks = smem_u32(sm.kv[stage_of(nidx)]);
-            if (act(0, j + 1)) {
-              issue_qk(tS[0], q_s[0], ks);
-              tc_commit(smem_u32(&sm.s_full[0]));
-            }
+            if (act(0, j + 1)) issue_s(0, j + 1, ks);
           }
-          // Tile 1: PV1(j), then S1(j+1).
-          if (act(1, j)) {
-            ok = mbar_wait(smem_u32(&sm.p_full[1]), it[1] & 1, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(tO[1], tS[1], vs, it[1] > 0);
-            ++it[1];
-            if (j == hi_t[1] - 1) tc_commit(smem_u32(&sm.o_full[1]));
-          }
+          if (act(1, j) && !(ok = issue_o(1, j, vs))) break;
           tc_commit(smem_u32(&sm.kv_empty[stage_of(vidx)]));
           if (has_next) {
-            if (act(1, j + 1)) {
-              issue_qk(tS[1], q_s[1], ks);
-              tc_commit(smem_u32(&sm.s_full[1]));
-            }
+            if (act(1, j + 1)) issue_s(1, j + 1, ks);
             tc_commit(smem_u32(&sm.kv_empty[stage_of(nidx)]));
           }
+          kvi += has_next ? 2 : 1;
         }
       }
       // All MMAs issued by this thread must complete before TMEM is freed.
@@ -279,38 +320,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int t = warp >> 2;  // query tile of this warpgroup
+    const int t = warp >> 2;  // query tile slot of this warpgroup
     const int wq = warp & 3;  // warp within the warpgroup -> TMEM lanes 32*wq..
     const int row = wq * 32 + lane;
-    const int row_g = r0[t] + row;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * 128;
     const float sl2 = args.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    int ns = 0;    // S tiles consumed (s_full phase)
+    int nout = 0;  // items finished (o_full phase)
     bool ok = true;
-    int it = 0;
-    if (t == 0 || has1) {
-      for (int j = lo_t[t]; j < hi_t[t]; ++j, ++it) {
-        ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), it & 1, abort_flag);
+    for (int k = 0; ok; ++k) {
+      const int lin = item_of(k, total);
+      if (lin < 0) break;
+      const Item item = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+      if (t == 1 && !item.has1) continue;
+      const int r0 = item.r0[t];
+      const int row_g = r0 + row;
+      float m = -INFINITY, l = 0.f;
+      bool nan_row = false;
+      for (int j = item.lo_t[t]; j < item.hi_t[t]; ++j, ++ns) {
+        ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), ns & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        uint32_t s[BN];
-        FA_TMEM_LD32(tS + 0, (s + 0));
-        FA_TMEM_LD32(tS + 32, (s + 32));
-        FA_TMEM_LD32(tS + 64, (s + 64));
-        FA_TMEM_LD32(tS + 96, (s + 96));
-        tmem_ld_wait();
-        if (tile_needs_mask(j, r0[t], n, args.causal, args.window)) {
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (!key_visible(row_g, j * BN + c, n, args.causal, args.window))
-              s[c] = __float_as_uint(-INFINITY);
+        const bool masked = tile_needs_mask(j, r0, n, args.causal, args.window);
+        // Visible columns of this row form one interval [c_lo, c_hi) (whole tile if unmasked).
+        int c_lo = 0, c_hi = BN;
+        if (masked) {
+          const int base = j * BN;
+          c_hi = min(BN, n - base);
+          if (args.causal) c_hi = min(c_hi, row_g - base + 1);
+          if (args.window > 0) c_lo = max(0, row_g - args.window + 1 - base);
         }
-        float mx = -INFINITY;
+        // Pass 1: the row max.  All 128 scores are loaded at once but only the max is
+        // kept; eight independent chains of 3-input max.  The max keeps NaN, so a NaN
+        // score marks the row (its output is NaN at the end).
+        float mx;
+        {
+          uint32_t s[BN];
+          FA_TMEM_LD32(tS + 0, (s + 0));
+          FA_TMEM_LD32(tS + 32, (s + 32));
+          FA_TMEM_LD32(tS + 64, (s + 64));
+          FA_TMEM_LD32(tS + 96, (s + 96));
+          tmem_ld_wait();
+          if (masked) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-        const float m_new = fmaxf(m, mx);
+            for (int c = 0; c < BN; ++c)
+              if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+          }
+          float mm[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mm[k] = fmax3_nan(__uint_as_float(s[k]), __uint_as_float(s[k + 8]), -INFINITY);
+#pragma unroll
+          for (int c = 16; c < BN; c += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              mm[k] = fmax3_nan(mm[k], __uint_as_float(s[c + k]), __uint_as_float(s[c + 8 + k]));
+          mx = fmax3_nan(fmax3_nan(mm[0], mm[1], mm[2]), fmax3_nan(mm[3], mm[4], mm[5]),
+                         fmax3_nan(mm[6], mm[7], -INFINITY));
+        }
+        nan_row |= (mx != mx);
+        const float m_new = fmaxf(m, mx);  // ignores a NaN mx
         // (m_new - m) is +inf on the first visible tile and NaN while the row is
         // still empty; only the former moves the reference max.
         const bool need = (m_new - m) * sl2 > kRescaleThreshold;
@@ -321,21 +392,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           l *= alpha;
         }
         const float ms = (m == -INFINITY) ? 0.f : m * sl2;
-        float rs = 0.f;
+        // Pass 2, 32 columns at a time with the next chunk's TMEM load in flight:
+        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> bf16 into TMEM.  P chunk c
+        // (16 columns at 16c) only overwrites S columns already read.  On unmasked
+        // tiles one pair in four takes the FMA-pipe polynomial instead of the
+        // special-function unit, which retires one ex2 warp-instruction per ~16
+        // cycles per sub-partition.
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+        uint32_t sc[2][32];
+        FA_TMEM_LD32(tS + 0, sc[0]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // P columns [32h, 32h + 32) hold keys [64h, 64h + 64); S there is already in registers.
-          uint32_t p[32];
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld_wait();
+          if (c + 1 < 4) FA_TMEM_LD32(tS + 32 * (c + 1), sc[(c + 1) & 1]);
+          uint32_t* x = sc[c & 1];
+          if (masked) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[64 * h + 2 * c]), sl2, -ms));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[64 * h + 2 * c + 1]), sl2, -ms));
-            rs += p0 + p1;
-            p[c] = pack_bf16x2(p0, p1);
+            for (int e = 0; e < 32; ++e)
+              if (32 * c + e < c_lo || 32 * c + e >= c_hi) x[e] = __float_as_uint(-INFINITY);
           }
-          FA_TMEM_ST32(tS + 32 * h, p);
+          uint32_t p[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = fmaf(__uint_as_float(x[e]), sl2, -ms);
+            const float x1 = fmaf(__uint_as_float(x[e + 1]), sl2, -ms);
+            float p0, p1;
+            if ((e & 6) == 6 && !masked) {
+              f2_unpack(exp2_poly_pair(f2_pack(x0, x1)), p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            if (e & 2) {
+              acc2 += p0;
+              acc3 += p1;
+            } else {
+              acc0 += p0;
+              acc1 += p1;
+            }
+            p[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+                  tS + 16 * c),
+              "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3]), "r"(p[4]), "r"(p[5]), "r"(p[6]), "r"(p[7]),
+              "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15])
+              : "memory");
         }
-        if (it > 0 && __any_sync(0xffffffffu, need)) {
+        const float rs = (acc0 + acc1) + (acc2 + acc3);
+        if (j > item.lo_t[t] && __any_sync(0xffffffffu, need)) {
           // O_t's last update (PV_t(j-1)) is complete: S_t(j) was issued after it.  The
           // rescale happens after P is stored (S is no longer live) and before p_full.
 #pragma unroll
@@ -353,34 +458,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(smem_u32(&sm.p_full[t]));
         l += rs;
       }
-      // Epilogue: O / l in bf16 and lse = m * scale + ln l.
-      if (ok && hi_t[t] > lo_t[t]) ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (!ok) break;
+      // Epilogue: O / l in bf16 and lse = m * scale + ln l.  O_t is read out first and
+      // released (o_free) so the next item's PV can start while the stores drain.
+      ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nout & 1, abort_flag);
+      if (!ok) break;
+      ++nout;
+      tc_fence_after();
+      uint32_t o[D];
+      FA_TMEM_LD32(tO + 0, (o + 0));
+      FA_TMEM_LD32(tO + 32, (o + 32));
+      FA_TMEM_LD32(tO + 64, (o + 64));
+      FA_TMEM_LD32(tO + 96, (o + 96));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.o_free[t]));
+      if (nan_row) l = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
+      const float inv = l > 0.f ? 1.f / l : (l == 0.f ? 0.f : l);
+      if (row_g < n) {
         __nv_bfloat16* orow =
-            reinterpret_cast<__nv_bfloat16*>(args.o) + (static_cast<size_t>(bh) * n + row_g) * D;
+            reinterpret_cast<__nv_bfloat16*>(args.o) + (static_cast<size_t>(item.bh) * n + row_g) * D;
+        uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          FA_TMEM_LD32(tO + 32 * c, r);
-          tmem_ld_wait();
-          if (row_g < n) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(r[8 * v4 + 0]) * inv, __uint_as_float(r[8 * v4 + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * inv, __uint_as_float(r[8 * v4 + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * inv, __uint_as_float(r[8 * v4 + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * inv, __uint_as_float(r[8 * v4 + 7]) * inv);
-              dst[v4] = w;
-            }
-          }
+        for (int v4 = 0; v4 < D / 8; ++v4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+          dst[v4] = w;
         }
-        if (row_g < n && args.lse != nullptr)
-          args.lse[static_cast<size_t>(bh) * n + row_g] =
-              l > 0.f ? m * args.scale + logf(l) : -INFINITY;
+        if (args.lse != nullptr)
+          args.lse[static_cast<size_t>(item.bh) * n + row_g] =
+              l > 0.f ? m * args.scale + logf(l) : (l == 0.f ? -INFINITY : l);
       }
     }
   }
@@ -404,10 +514,13 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fwd_tc_kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int num_pairs = (a.N + 2 * BM - 1) / (2 * BM);
-  const long long grid = static_cast<long long>(num_pairs) * a.B * a.H;
-  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-  fwd_tc_kernel<<<static_cast<unsigned>(grid), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, a);
+  const long long items = static_cast<long long>((a.N + 2 * BM - 1) / (2 * BM)) * a.B * a.H;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  int sms = 0;
+  e = sm_count(&sms);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
+  fwd_tc_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

@@ -62,6 +62,8 @@ bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_
                          long long heads, int box_rows);
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device and kernel.
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
+// Number of SMs of the current device (cached per device).
+cudaError_t sm_count(int* out);
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);
