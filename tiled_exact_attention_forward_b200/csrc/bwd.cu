@@ -79,10 +79,6 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int count) {  // bar.sync id, count
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
 __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);

@@ -80,6 +80,11 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
   return __all_sync(0xffffffffu, ok);
 }
 
+// Barrier of `nthreads` threads (whole warps) on named barrier `id` (1..15).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // AND of `v` over the `nthreads` threads (whole warps) that use named barrier `id`.
 __device__ __forceinline__ bool named_bar_all(bool v, int id, int nthreads) {
   uint32_t r;

@@ -46,9 +46,10 @@ constexpr int D = 128;                  // head dimension
 constexpr int NS = 4;                   // K/V ring stages (K and V tiles interleaved)
 constexpr int TILE_BYTES = BM * D * 2;  // one 128 x 128 bf16 tile = 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;  // one 64-column half (a 128-byte-swizzled box)
-constexpr int NUM_THREADS = 320;
-constexpr int MMA_WARP = 8;
-constexpr int TMA_WARP = 9;
+constexpr int NUM_THREADS = 576;     // 16 softmax warps + MMA warp + TMA warp
+constexpr int WG_THREADS = 256;      // one softmax warpgroup pair per query tile
+constexpr int MMA_WARP = 16;
+constexpr int TMA_WARP = 17;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Smem {
@@ -64,6 +65,10 @@ struct Smem {
   uint64_t o_full[2];
   uint64_t o_free[2];
   uint64_t mma_done;
+  // Row statistics exchanged between the two threads of a row (column halves):
+  // [tile][step parity][half][row].
+  float xmax[2][2][2][BM];
+  float xsum[2][2][BM];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -104,8 +109,10 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
     // V tile: [64-column half][128 keys][64 cols]; a K step of 16 keys = 16 rows.
+    // P of keys [64h, 64h + 64) sits in S columns [64h, 64h + 32) (bf16 pairs).
     const uint64_t b = smem_desc_sw128(v_smem + kk * 16 * 128, HALF_BYTES, 1024);
-    mma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    const uint32_t a_col = (kk >> 2) * 64 + (kk & 3) * 8;
+    mma_ts(d_tmem, p_tmem + a_col, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -167,9 +174,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&sm.q_full[t]), 1);
       mbar_init(smem_u32(&sm.q_empty[t]), 1);
       mbar_init(smem_u32(&sm.s_full[t]), 1);
-      mbar_init(smem_u32(&sm.p_full[t]), BM);
+      mbar_init(smem_u32(&sm.p_full[t]), WG_THREADS);
       mbar_init(smem_u32(&sm.o_full[t]), 1);
-      mbar_init(smem_u32(&sm.o_free[t]), BM);
+      mbar_init(smem_u32(&sm.o_free[t]), WG_THREADS);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), 1);
@@ -319,13 +326,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int t = warp >> 2;  // query tile slot of this warpgroup
-    const int wq = warp & 3;  // warp within the warpgroup -> TMEM lanes 32*wq..
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    // ------------------------------------------------------------ softmax warps
+    // 8 warps per query tile: warp i of the tile reads TMEM lanes 32*(i%4).. (one row
+    // per thread) and columns [64h, 64h + 64) with h = i/4, so two threads share a
+    // row and exchange its max and sum through shared memory.
+    const int t = warp >> 3;         // query tile slot
+    const int wi = warp & 7;
+    const int hc = wi >> 2;          // column half
+    const int row = (wi & 3) * 32 + lane;
+    const int bar_id = 1 + t;        // named barrier of this tile's 256 threads
+    const uint32_t lane_off = static_cast<uint32_t>((wi & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128 + 64 * hc;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128 + 64 * hc;
     const float sl2 = args.scale_log2;
     int ns = 0;    // S tiles consumed (s_full phase)
     int nout = 0;  // items finished (o_full phase)
@@ -337,53 +349,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (t == 1 && !item.has1) continue;
       const int r0 = item.r0[t];
       const int row_g = r0 + row;
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
       bool nan_row = false;
       for (int j = item.lo_t[t]; j < item.hi_t[t]; ++j, ++ns) {
         ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), ns & 1, abort_flag);
-        if (!ok) break;
         tc_fence_after();
+        uint32_t s[64];
+        FA_TMEM_LD32(tS + 0, (s + 0));
+        FA_TMEM_LD32(tS + 32, (s + 32));
+        tmem_ld_wait();
         const bool masked = tile_needs_mask(j, r0, n, args.causal, args.window);
-        // Visible columns of this row form one interval [c_lo, c_hi) (whole tile if unmasked).
-        int c_lo = 0, c_hi = BN;
         if (masked) {
-          const int base = j * BN;
-          c_hi = min(BN, n - base);
+          // Visible keys of this row form one interval; columns of this half are 64h + c.
+          const int base = j * BN + 64 * hc;
+          int c_hi = min(64, n - base);
           if (args.causal) c_hi = min(c_hi, row_g - base + 1);
-          if (args.window > 0) c_lo = max(0, row_g - args.window + 1 - base);
+          const int c_lo = args.window > 0 ? max(0, row_g - args.window + 1 - base) : 0;
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
         }
-        // Pass 1: the row max.  All 128 scores are loaded at once but only the max is
-        // kept; eight independent chains of 3-input max.  The max keeps NaN, so a NaN
-        // score marks the row (its output is NaN at the end).
-        float mx;
-        {
-          uint32_t s[BN];
-          FA_TMEM_LD32(tS + 0, (s + 0));
-          FA_TMEM_LD32(tS + 32, (s + 32));
-          FA_TMEM_LD32(tS + 64, (s + 64));
-          FA_TMEM_LD32(tS + 96, (s + 96));
-          tmem_ld_wait();
-          if (masked) {
+        // Half-row max: eight chains of 3-input max; NaN-propagating so a NaN score
+        // marks the row (its output is NaN at the end).
+        float mm[8];
 #pragma unroll
-            for (int c = 0; c < BN; ++c)
-              if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
-          }
-          float mm[8];
+        for (int q = 0; q < 8; ++q)
+          mm[q] = fmax3_nan(__uint_as_float(s[q]), __uint_as_float(s[q + 8]), -INFINITY);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mm[k] = fmax3_nan(__uint_as_float(s[k]), __uint_as_float(s[k + 8]), -INFINITY);
+        for (int c = 16; c < 64; c += 16)
 #pragma unroll
-          for (int c = 16; c < BN; c += 16)
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              mm[k] = fmax3_nan(mm[k], __uint_as_float(s[c + k]), __uint_as_float(s[c + 8 + k]));
-          mx = fmax3_nan(fmax3_nan(mm[0], mm[1], mm[2]), fmax3_nan(mm[3], mm[4], mm[5]),
-                         fmax3_nan(mm[6], mm[7], -INFINITY));
-        }
+          for (int q = 0; q < 8; ++q)
+            mm[q] = fmax3_nan(mm[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
+        const float hm = fmax3_nan(fmax3_nan(mm[0], mm[1], mm[2]), fmax3_nan(mm[3], mm[4], mm[5]),
+                                   fmax3_nan(mm[6], mm[7], -INFINITY));
+        sm.xmax[t][ns & 1][hc][row] = hm;
+        // Barrier of the tile's 256 threads: both halves' maxima are visible, and the
+        // whole group agrees on whether to go on.
+        ok = named_bar_all(ok, bar_id, WG_THREADS);
+        if (!ok) break;
+        const float mx = fmax3_nan(hm, sm.xmax[t][ns & 1][hc ^ 1][row], -INFINITY);
         nan_row |= (mx != mx);
         const float m_new = fmaxf(m, mx);  // ignores a NaN mx
         // (m_new - m) is +inf on the first visible tile and NaN while the row is
-        // still empty; only the former moves the reference max.
+        // still empty; only the former moves the reference max.  Both halves of a
+        // row take the same decision from the same numbers.
         const bool need = (m_new - m) * sl2 > kRescaleThreshold;
         float alpha = 1.f;
         if (need) {
@@ -392,37 +401,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           l *= alpha;
         }
         const float ms = (m == -INFINITY) ? 0.f : m * sl2;
-        // Pass 2, 32 columns at a time with the next chunk's TMEM load in flight:
-        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> bf16 into TMEM.  P chunk c
-        // (16 columns at 16c) only overwrites S columns already read.  On unmasked
-        // tiles one pair in four takes the FMA-pipe polynomial instead of the
-        // special-function unit, which retires one ex2 warp-instruction per ~16
-        // cycles per sub-partition.
+        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> bf16 pairs over this
+        // half's first 32 S columns (already read).
         float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-        uint32_t sc[2][32];
-        FA_TMEM_LD32(tS + 0, sc[0]);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld_wait();
-          if (c + 1 < 4) FA_TMEM_LD32(tS + 32 * (c + 1), sc[(c + 1) & 1]);
-          uint32_t* x = sc[c & 1];
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (32 * c + e < c_lo || 32 * c + e >= c_hi) x[e] = __float_as_uint(-INFINITY);
-          }
+        for (int c = 0; c < 2; ++c) {
           uint32_t p[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(__uint_as_float(x[e]), sl2, -ms);
-            const float x1 = fmaf(__uint_as_float(x[e + 1]), sl2, -ms);
-            float p0, p1;
-            if ((e & 6) == 6 && !masked) {
-              f2_unpack(exp2_poly_pair(f2_pack(x0, x1)), p0, p1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            const float p0 = ex2_approx(fmaf(__uint_as_float(s[32 * c + e]), sl2, -ms));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(s[32 * c + e + 1]), sl2, -ms));
             if (e & 2) {
               acc2 += p0;
               acc3 += p1;
@@ -439,12 +427,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15])
               : "memory");
         }
-        const float rs = (acc0 + acc1) + (acc2 + acc3);
         if (j > item.lo_t[t] && __any_sync(0xffffffffu, need)) {
-          // O_t's last update (PV_t(j-1)) is complete: S_t(j) was issued after it.  The
-          // rescale happens after P is stored (S is no longer live) and before p_full.
+          // O_t's last update (PV_t(j-1)) is complete: S_t(j) was issued after it.
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
             FA_TMEM_LD32(tO + 32 * c, r);
             tmem_ld_wait();
@@ -456,31 +442,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sm.p_full[t]));
-        l += rs;
+        l += (acc0 + acc1) + (acc2 + acc3);
       }
       if (!ok) break;
       // Epilogue: O / l in bf16 and lse = m * scale + ln l.  O_t is read out first and
       // released (o_free) so the next item's PV can start while the stores drain.
       ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nout & 1, abort_flag);
-      if (!ok) break;
       ++nout;
       tc_fence_after();
-      uint32_t o[D];
+      uint32_t o[64];
       FA_TMEM_LD32(tO + 0, (o + 0));
       FA_TMEM_LD32(tO + 32, (o + 32));
-      FA_TMEM_LD32(tO + 64, (o + 64));
-      FA_TMEM_LD32(tO + 96, (o + 96));
       tmem_ld_wait();
       tc_fence_before();
+      sm.xsum[t][hc][row] = l;
+      ok = named_bar_all(ok, bar_id, WG_THREADS);
       mbar_arrive(smem_u32(&sm.o_free[t]));
-      if (nan_row) l = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
-      const float inv = l > 0.f ? 1.f / l : (l == 0.f ? 0.f : l);
+      if (!ok) break;
+      float lt = l + sm.xsum[t][hc ^ 1][row];
+      // The sums may be read again only after the next item's first exchange barrier.
+      if (nan_row) lt = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
+      const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
       if (row_g < n) {
-        __nv_bfloat16* orow =
-            reinterpret_cast<__nv_bfloat16*>(args.o) + (static_cast<size_t>(item.bh) * n + row_g) * D;
+        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
+                              (static_cast<size_t>(item.bh) * n + row_g) * D + 64 * hc;
         uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-        for (int v4 = 0; v4 < D / 8; ++v4) {
+        for (int v4 = 0; v4 < 8; ++v4) {
           uint4 w;
           w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
           w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
@@ -488,9 +476,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
           dst[v4] = w;
         }
-        if (args.lse != nullptr)
+        if (hc == 0 && args.lse != nullptr)
           args.lse[static_cast<size_t>(item.bh) * n + row_g] =
-              l > 0.f ? m * args.scale + logf(l) : (l == 0.f ? -INFINITY : l);
+              lt > 0.f ? m * args.scale + logf(lt) : (lt == 0.f ? -INFINITY : lt);
       }
     }
   }
