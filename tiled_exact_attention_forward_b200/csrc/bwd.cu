@@ -11,16 +11,18 @@
 // Kernels: bwd_pre (D and zeroed fp32 dQ accumulator), bwd_main (below),
 // bwd_post (dQ fp32 -> bf16).
 //
-// bwd_main, one CTA per (batch*head, 128-key tile), 320 threads:
-//   * warp 9 loads K and V once, then (Q_i, dO_i) pairs by TMA into a
+// bwd_main, one CTA per (batch*head, 128-key tile), 576 threads:
+//   * warp 17 loads K and V once, then (Q_i, dO_i) pairs by TMA into a
 //     two-stage ring;
-//   * warp 8 allocates tensor memory and issues the MMAs from one thread;
-//   * warps 0-3 (one thread per key row = one TMEM lane) turn S^T, dP^T into
-//     P^T and dS^T: bf16 back into tensor memory (operands of the dV and dK
-//     MMAs) and dS^T into shared memory (operand of the dQ MMA);
-//   * warps 4-7 (one thread per query row) read dQ_i out of tensor memory
-//     and add it into the fp32 accumulator with vector reductions; at the
-//     end warps 0-3 write dV and warps 4-7 write dK.
+//   * warp 16 allocates tensor memory and issues the MMAs from one thread;
+//   * warps 0-7 turn S^T, dP^T into P^T and dS^T: warp w handles the key rows
+//     of TMEM lane quarter w%4 and the query columns [64h, 64h + 64),
+//     h = w/4 -- two threads per key row.  P^T and dS^T go back into tensor
+//     memory as bf16 (operands of the dV and dK MMAs) and dS^T also into
+//     shared memory (operand of the dQ MMA);
+//   * warps 8-15 read dQ_i out of tensor memory (two threads per query row,
+//     64 columns each) and add it into the fp32 accumulator with vector
+//     reductions; at the end warps 0-7 write dV and warps 8-15 write dK.
 // Tensor memory (512 columns): [S^T -> P^T, later dQ_i] [dP^T -> dS^T] [dV] [dK].
 // Keys are the MMA rows of S^T = K Q^T and dP^T = V dO^T, so P^T and dS^T
 // land with keys on lanes -- exactly the A operands dV and dK need.
@@ -35,9 +37,10 @@ constexpr int BQ = 128;  // queries per inner tile
 constexpr int D = 128;
 constexpr int TILE_BYTES = 128 * D * 2;
 constexpr int HALF_BYTES = TILE_BYTES / 2;
-constexpr int NUM_THREADS = 320;
-constexpr int MMA_WARP = 8;
-constexpr int TMA_WARP = 9;
+constexpr int NUM_THREADS = 576;
+constexpr int GROUP = 256;  // threads of the P/dS group and of the dQ group
+constexpr int MMA_WARP = 16;
+constexpr int TMA_WARP = 17;
 
 struct Smem {
   uint8_t k[TILE_BYTES];
@@ -91,13 +94,14 @@ __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint
 }
 
 // D[128 x d] (+)= A[tmem, 128 x 128 bf16] * B, B = [128 rows (K)][d] tile (MN-major).
+// A's K columns [64h, 64h + 64) (bf16 pairs) sit at TMEM columns [64h, 64h + 32).
 __device__ __forceinline__ void issue_tmemA_b(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
                                               bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8,
+           smem_desc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem).
@@ -139,9 +143,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.dp_full), 1);
-    mbar_init(smem_u32(&sm.ds_ready), 128);
+    mbar_init(smem_u32(&sm.ds_ready), GROUP);
     mbar_init(smem_u32(&sm.dq_full), 1);
-    mbar_init(smem_u32(&sm.dq_free), 128);
+    mbar_init(smem_u32(&sm.dq_free), GROUP);
     mbar_init(smem_u32(&sm.acc_done), 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -222,72 +226,86 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait_drain(smem_u32(&sm.acc_done), 0);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // -------------------------------------------------- P^T and dS^T (thread = key row)
-    const int row = warp * 32 + lane;
+  } else if (warp < 8) {
+    // -------------------------------------------------- P^T and dS^T (thread = key row x 64 queries)
+    const int hc = warp >> 2;
+    const int row = (warp & 3) * 32 + lane;
     const int key = kt * BM + row;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + T_S, tDP = tmem + lane_off + T_DP;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + T_S + 64 * hc, tDP = tmem + lane_off + T_DP + 64 * hc;
     const float sl2 = args.scale_log2;
     const float* lse_g = args.lse + static_cast<size_t>(bh) * n;
     const float* del_g = args.ws_delta + static_cast<size_t>(bh) * n;
-    uint8_t* ds_row = sm.ds + row * 128;
+    uint8_t* ds_row = sm.ds + hc * HALF_BYTES + row * 128;
+    const int gt = threadIdx.x;  // 0..255: loads row statistic gt & 127 (lse if < 128, else D)
     bool ok = true;
     // Prefetch the first tile's row statistics.
-    float lse_next = INFINITY, del_next = 0.f;
-    if (nq > 0) {
-      const int qi = qlo * BQ + row;
-      if (qi < n) {
-        const float l = lse_g[qi];
-        lse_next = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-        del_next = del_g[qi];
-      }
-    }
-    for (int idx = 0; idx < nq; ++idx) {
-      const int s = idx & 1;
-      sm.lse2[s][row] = lse_next;
-      sm.delta[s][row] = del_next;
-      named_bar_sync(1, 128);
-      if (idx + 1 < nq) {
-        const int qi = (qlo + idx + 1) * BQ + row;
-        lse_next = INFINITY;
-        del_next = 0.f;
+    float stat_next = 0.f;
+    auto load_stat = [&](int qt) {
+      const int qi = qt * BQ + (gt & 127);
+      if (gt < 128) {
+        float v = INFINITY;  // past N: P = 2^(-inf) = 0
         if (qi < n) {
           const float l = lse_g[qi];
-          lse_next = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-          del_next = del_g[qi];
+          v = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
         }
+        return v;
       }
+      return qi < n ? del_g[qi] : 0.f;
+    };
+    if (nq > 0) stat_next = load_stat(qlo);
+    for (int idx = 0; idx < nq; ++idx) {
+      const int s = idx & 1;
+      if (gt < 128) sm.lse2[s][gt] = stat_next; else sm.delta[s][gt - 128] = stat_next;
+      named_bar_sync(1, GROUP);
+      if (idx + 1 < nq) stat_next = load_stat(qlo + idx + 1);
       const int qt = qlo + idx;
       const bool masked = tile_needs_mask(kt, qt, n, args.causal, args.window);
       ok = mbar_wait(smem_u32(&sm.s_full), idx & 1, abort_flag);
       if (ok) ok = mbar_wait(smem_u32(&sm.dp_full), idx & 1, abort_flag);
-      // One decision for the whole warpgroup: it meets at named barrier 1 every step.
-      ok = named_bar_all(ok, 2, 128);
+      // One decision for the whole group: it meets at named barrier 1 every step.
+      ok = named_bar_all(ok, 2, GROUP);
       if (!ok) break;
       tc_fence_after();
+      // Visible queries of this key row form one interval [q_lo, q_hi) of this half.
+      int q_lo = 0, q_hi = 64;
+      if (masked) {
+        const int qbase = qt * BQ + 64 * hc;
+        if (args.causal) q_lo = max(0, key - qbase);
+        if (args.window > 0) q_hi = min(64, key + args.window - qbase);
+        q_hi = min(q_hi, n - qbase);  // queries past N have lse2 = +inf anyway
+        if (key >= n) q_hi = 0;
+      }
+      const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][64 * hc]);
+      const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[s][64 * hc]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t sr[32], dr[32];
         FA_TMEM_LD32(tS + 32 * c, sr);
         FA_TMEM_LD32(tDP + 32 * c, dr);
         tmem_ld_wait();
         uint32_t pp[16], dd[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -sm.lse2[s][32 * c + e]));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), sl2, -sm.lse2[s][32 * c + e + 1]));
-          if (masked) {
-            const int q0 = qt * BQ + 32 * c + e;
-            if (!key_visible(q0, key, n, args.causal, args.window)) p0 = 0.f;
-            if (!key_visible(q0 + 1, key, n, args.causal, args.window)) p1 = 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 lv = l4[8 * c + e4];
+          const float4 dv = d4[8 * c + e4];
+          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+          const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = 4 * e4 + u;
+            float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lq[u]));
+            if (masked && (32 * c + e < q_lo || 32 * c + e >= q_hi)) p = 0.f;
+            pv[u] = p;
+            dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
           }
-          const float d0 = p0 * (__uint_as_float(dr[e]) - sm.delta[s][32 * c + e]);
-          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - sm.delta[s][32 * c + e + 1]);
-          pp[e >> 1] = pack_bf16x2(p0, p1);
-          dd[e >> 1] = pack_bf16x2(d0, d1);
+          pp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+          pp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dd[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
+          dd[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        // P^T over S^T columns [16c, 16c+16), dS^T over dP^T columns (both already read).
+        // P^T over S^T columns [64h + 16c, +16), dS^T over dP^T columns (both already read).
         asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
                 tS + 16 * c),
@@ -302,12 +320,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             "r"(dd[8]), "r"(dd[9]), "r"(dd[10]), "r"(dd[11]), "r"(dd[12]), "r"(dd[13]), "r"(dd[14]),
             "r"(dd[15])
             : "memory");
-        // dS (queries 32c..32c+31 of this key row) into the swizzled MN-major tile.
-        uint8_t* half = ds_row + (c >> 1) * HALF_BYTES;
+        // dS (queries 64h + 32c .. +31 of this key row) into the swizzled MN-major tile.
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int chunk = ((c & 1) * 4 + u) ^ (row & 7);
-          *reinterpret_cast<uint4*>(half + chunk * 16) =
+          const int chunk = (c * 4 + u) ^ (row & 7);
+          *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
               make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
         }
       }
@@ -316,16 +333,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.ds_ready));
     }
-    // Epilogue: dV rows.
+    // Epilogue: dV rows (64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
     if (ok) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         if (nq > 0) {
-          FA_TMEM_LD32(tmem + lane_off + T_DV + 32 * c, r);
+          FA_TMEM_LD32(tmem + lane_off + T_DV + 64 * hc + 32 * c, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -343,10 +360,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // -------------------------------------------------- dQ read-out (thread = query row)
-    const int wq = warp & 3;
-    const int row = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    // -------------------------------------------------- dQ read-out (thread = query row x 64 columns)
+    const int hc = (warp - 8) >> 2;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = args.scale;
     bool ok = true;
     for (int idx = 0; idx < nq; ++idx) {
@@ -354,34 +371,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const int qi = (qlo + idx) * BQ + row;
-      float* acc = args.ws_dq + (static_cast<size_t>(bh) * n + qi) * D;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        FA_TMEM_LD32(tmem + lane_off + T_S + 32 * c, r);
-        tmem_ld_wait();
-        if (qi < n) {
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            red_add_v4(acc + 32 * c + 4 * v4, __uint_as_float(r[4 * v4]) * scale,
-                       __uint_as_float(r[4 * v4 + 1]) * scale, __uint_as_float(r[4 * v4 + 2]) * scale,
-                       __uint_as_float(r[4 * v4 + 3]) * scale);
-        }
-      }
+      float* acc = args.ws_dq + (static_cast<size_t>(bh) * n + qi) * D + 64 * hc;
+      uint32_t r[64];
+      FA_TMEM_LD32(tmem + lane_off + T_S + 64 * hc, r);
+      FA_TMEM_LD32(tmem + lane_off + T_S + 64 * hc + 32, (r + 32));
+      tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.dq_free));
+      mbar_arrive(smem_u32(&sm.dq_free));  // TMEM read: the next S^T may overwrite it
+      if (qi < n) {
+#pragma unroll
+        for (int v4 = 0; v4 < 16; ++v4)
+          red_add_v4(acc + 4 * v4, __uint_as_float(r[4 * v4]) * scale, __uint_as_float(r[4 * v4 + 1]) * scale,
+                     __uint_as_float(r[4 * v4 + 2]) * scale, __uint_as_float(r[4 * v4 + 3]) * scale);
+      }
     }
-    // Epilogue: dK rows (scaled).
+    // Epilogue: dK rows (scaled, 64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
     const int key = kt * BM + row;
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
     if (ok) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         if (nq > 0) {
-          FA_TMEM_LD32(tmem + lane_off + T_DK + 32 * c, r);
+          FA_TMEM_LD32(tmem + lane_off + T_DK + 64 * hc + 32 * c, r);
           tmem_ld_wait();
         } else {
 #pragma unroll
