@@ -21,8 +21,11 @@
 //     memory as bf16 (operands of the dV and dK MMAs) and dS^T also into
 //     shared memory (operand of the dQ MMA);
 //   * warps 8-15 read dQ_i out of tensor memory (two threads per query row,
-//     64 columns each) and add it into the fp32 accumulator with vector
-//     reductions; at the end warps 0-7 write dV and warps 8-15 write dK.
+//     64 columns each), stage it in shared memory (the dS buffer, free once
+//     the dQ MMA has read it) and add it into the fp32 accumulator with TMA
+//     bulk reduce-adds, so no per-thread global atomics compete with the
+//     P/dS warps' shared-memory traffic; at the end warps 0-7 write dV and
+//     warps 8-15 write dK.
 // Tensor memory (512 columns): [S^T -> P^T, later dQ_i] [dP^T -> dS^T] [dV] [dK].
 // Keys are the MMA rows of S^T = K Q^T and dP^T = V dO^T, so P^T and dS^T
 // land with keys on lanes -- exactly the A operands dV and dK need.
@@ -54,6 +57,7 @@ struct Smem {
   uint64_t qdo_full[2];
   uint64_t qdo_empty[2];
   uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
+  uint64_t stage_free;  // dQ staging (in the dS buffer) read by the TMA (dQ group -> P/dS group)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -116,7 +120,7 @@ __device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_smem, uint
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tm_dq, BwdArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusTimeout);
@@ -147,6 +151,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&sm.dq_full), 1);
     mbar_init(smem_u32(&sm.dq_free), GROUP);
     mbar_init(smem_u32(&sm.acc_done), 1);
+    mbar_init(smem_u32(&sm.stage_free), 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -278,17 +283,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][64 * hc]);
       const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[s][64 * hc]);
+      // 16 query columns per step keeps S^T, dP^T and both outputs in registers.
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sr[32], dr[32];
-        FA_TMEM_LD32(tS + 32 * c, sr);
-        FA_TMEM_LD32(tDP + 32 * c, dr);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[16], dr[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(sr[0]), "=r"(sr[1]), "=r"(sr[2]), "=r"(sr[3]), "=r"(sr[4]), "=r"(sr[5]), "=r"(sr[6]), "=r"(sr[7]),
+              "=r"(sr[8]), "=r"(sr[9]), "=r"(sr[10]), "=r"(sr[11]), "=r"(sr[12]), "=r"(sr[13]), "=r"(sr[14]), "=r"(sr[15])
+            : "r"(tS + 16 * c));
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(dr[0]), "=r"(dr[1]), "=r"(dr[2]), "=r"(dr[3]), "=r"(dr[4]), "=r"(dr[5]), "=r"(dr[6]), "=r"(dr[7]),
+              "=r"(dr[8]), "=r"(dr[9]), "=r"(dr[10]), "=r"(dr[11]), "=r"(dr[12]), "=r"(dr[13]), "=r"(dr[14]), "=r"(dr[15])
+            : "r"(tDP + 16 * c));
         tmem_ld_wait();
-        uint32_t pp[16], dd[16];
+        uint32_t pp[8], dd[8];
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 lv = l4[8 * c + e4];
-          const float4 dv = d4[8 * c + e4];
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 lv = l4[4 * c + e4];
+          const float4 dv = d4[4 * c + e4];
           const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
           const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
           float pv[4], dsv[4];
@@ -296,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int u = 0; u < 4; ++u) {
             const int e = 4 * e4 + u;
             float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lq[u]));
-            if (masked && (32 * c + e < q_lo || 32 * c + e >= q_hi)) p = 0.f;
+            if (masked && (16 * c + e < q_lo || 16 * c + e >= q_hi)) p = 0.f;
             pv[u] = p;
             dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
           }
@@ -305,25 +319,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           dd[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
           dd[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        // P^T over S^T columns [64h + 16c, +16), dS^T over dP^T columns (both already read).
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-                tS + 16 * c),
-            "r"(pp[0]), "r"(pp[1]), "r"(pp[2]), "r"(pp[3]), "r"(pp[4]), "r"(pp[5]), "r"(pp[6]), "r"(pp[7]),
-            "r"(pp[8]), "r"(pp[9]), "r"(pp[10]), "r"(pp[11]), "r"(pp[12]), "r"(pp[13]), "r"(pp[14]),
-            "r"(pp[15])
-            : "memory");
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-                tDP + 16 * c),
-            "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7]),
-            "r"(dd[8]), "r"(dd[9]), "r"(dd[10]), "r"(dd[11]), "r"(dd[12]), "r"(dd[13]), "r"(dd[14]),
-            "r"(dd[15])
-            : "memory");
-        // dS (queries 64h + 32c .. +31 of this key row) into the swizzled MN-major tile.
+        // P^T over S^T columns [64h + 8c, +8), dS^T over dP^T columns (both already read).
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tS + 8 * c),
+                     "r"(pp[0]), "r"(pp[1]), "r"(pp[2]), "r"(pp[3]), "r"(pp[4]), "r"(pp[5]), "r"(pp[6]), "r"(pp[7])
+                     : "memory");
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tDP + 8 * c),
+                     "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7])
+                     : "memory");
+        // dS (queries 64h + 16c .. +15 of this key row) into the swizzled MN-major tile.
+        // The buffer doubles as the previous step's dQ staging: wait until the TMA has
+        // read that out (usually long done).
+        if (c == 0 && idx > 0) ok = mbar_wait_warp(smem_u32(&sm.stage_free), (idx - 1) & 1, abort_flag) && ok;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = (c * 4 + u) ^ (row & 7);
+        for (int u = 0; u < 2; ++u) {
+          const int chunk = (c * 2 + u) ^ (row & 7);
           *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
               make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
         }
@@ -365,26 +374,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float scale = args.scale;
+    const int gt = threadIdx.x - 256;  // 0..255 within the dQ group
     bool ok = true;
     for (int idx = 0; idx < nq; ++idx) {
       ok = mbar_wait_warp(smem_u32(&sm.dq_full), idx & 1, abort_flag);
-      if (!ok) break;
       tc_fence_after();
-      const int qi = (qlo + idx) * BQ + row;
-      float* acc = args.ws_dq + (static_cast<size_t>(bh) * n + qi) * D + 64 * hc;
+      const int q0 = (qlo + idx) * BQ;
       uint32_t r[64];
       FA_TMEM_LD32(tmem + lane_off + T_S + 64 * hc, r);
       FA_TMEM_LD32(tmem + lane_off + T_S + 64 * hc + 32, (r + 32));
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));  // TMEM read: the next S^T may overwrite it
-      if (qi < n) {
+      // Stage through the 32 KiB dS buffer in two rounds (column half 0, then 1):
+      // two 32-column x 128-row float boxes, 128-byte swizzled, reduced into the
+      // fp32 accumulator by the TMA (rows past N are skipped by the TMA).
+      for (int round = 0; round < 2; ++round) {
+        if (hc == round && ok) {
 #pragma unroll
-        for (int v4 = 0; v4 < 16; ++v4)
-          red_add_v4(acc + 4 * v4, __uint_as_float(r[4 * v4]) * scale, __uint_as_float(r[4 * v4 + 1]) * scale,
-                     __uint_as_float(r[4 * v4 + 2]) * scale, __uint_as_float(r[4 * v4 + 3]) * scale);
+          for (int b = 0; b < 2; ++b) {
+            uint8_t* box = sm.ds + b * (BQ * 128) + row * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const int e = 32 * b + 4 * ch;
+              *reinterpret_cast<float4*>(box + ((ch ^ (row & 7)) * 16)) =
+                  make_float4(__uint_as_float(r[e]) * scale, __uint_as_float(r[e + 1]) * scale,
+                              __uint_as_float(r[e + 2]) * scale, __uint_as_float(r[e + 3]) * scale);
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        ok = named_bar_all(ok, 3, GROUP);
+        if (gt == 0 && ok) {
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.ds), 64 * round, q0, bh);
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.ds) + BQ * 128, 64 * round + 32, q0, bh);
+          bulk_commit();
+          bulk_wait_read0();  // the staging may be rewritten once the TMA has read it
+        }
+        ok = named_bar_all(ok, 3, GROUP);
       }
+      if (gt == 0) mbar_arrive(smem_u32(&sm.stage_free));
+      if (!ok) break;
     }
+    if (gt == 0) bulk_wait0();  // every reduce-add has landed before the CTA ends
     // Epilogue: dK rows (scaled, 64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
     const int key = kt * BM + row;
@@ -462,9 +494,10 @@ cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   using namespace bwd;
   const long long bh = static_cast<long long>(a.B) * a.H;
   const long long rows = bh * a.N;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_tmap_bf16_rows(&tq, a.q, D, a.N, bh, BQ) || !make_tmap_bf16_rows(&tk, a.k, D, a.N, bh, BM) ||
-      !make_tmap_bf16_rows(&tv, a.v, D, a.N, bh, BM) || !make_tmap_bf16_rows(&tdo, a.dout, D, a.N, bh, BQ))
+      !make_tmap_bf16_rows(&tv, a.v, D, a.N, bh, BM) || !make_tmap_bf16_rows(&tdo, a.dout, D, a.N, bh, BQ) ||
+      !make_tmap_f32_rows(&tdq, a.ws_dq, D, a.N, bh, 32, BQ))
     return cudaErrorInvalidValue;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(bwd_main_kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
@@ -474,7 +507,7 @@ cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long nkt = (a.N + BM - 1) / BM;
-  bwd_main_kernel<<<static_cast<unsigned>(nkt * bh), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+  bwd_main_kernel<<<static_cast<unsigned>(nkt * bh), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long n8 = rows * D / 8;

@@ -46,6 +46,23 @@ bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_rows(void* map, const void* base, int d, long long rows_per_head, long long heads,
+                        int box_cols, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows_per_head),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                           static_cast<cuuint64_t>(d) * 4 * static_cast<cuuint64_t>(rows_per_head)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                  const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes) {
   // One bit per (device, kernel) pair; the kernel set is tiny and fixed.
   static std::mutex mu;

@@ -60,6 +60,9 @@ inline int decode_max_chunks(int cap) { return (cap + kDecodeChunk - 1) / kDecod
 // columns x box_rows rows, 128-byte swizzle, rows past the end read as zero.
 bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_head,
                          long long heads, int box_rows);
+// The same over a float32 array, boxes of box_cols (32: 128 bytes) x box_rows.
+bool make_tmap_f32_rows(void* map, const void* base, int d, long long rows_per_head,
+                        long long heads, int box_cols, int box_rows);
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device and kernel.
 cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
 // Number of SMs of the current device (cached per device).
