@@ -85,14 +85,15 @@ def source_hash(names):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, sources):
-    """DRAM bytes per launch from the committed ncu summary, if it is current."""
+def profiled_traffic(kernel: str, workload: str, sources):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary (profiles/dram_traffic.json), if its kernel source is current."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel)
+    e = d.get(f"{kernel}@{workload}")
     if not e or e.get("source_hash") != source_hash(sources):
         return None
     return e.get("bytes_per_launch")
@@ -349,7 +350,7 @@ def run_gpu(args, rank, world, local_rank):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_kind} ({'copy bandwidth' if unit == 'GB/s' else 'cuBLAS bf16 burst'})"
     roof["kernel"] = kernel
-    roof["traffic"] = profiled_traffic(kernel, sources)
+    roof["traffic"] = profiled_traffic(kernel, w.name, sources)
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
