@@ -16,10 +16,20 @@
 //     or window mask hides from every row of a query tile are never loaded
 //     for it; only tiles that straddle a mask edge (or the ragged end of the
 //     sequence) get the per-element mask.
-//   * Warp roles (320 threads): warps 0-3 and 4-7 are two softmax
-//     warpgroups, one per query tile (thread = one query row = one TMEM
-//     lane); warp 8 allocates tensor memory and issues every MMA from one
-//     thread; warp 9 issues the TMA loads.
+//   * Warp roles (608 threads): warps 0-7 and 8-15 are the softmax warps of
+//     query tiles 0 and 1 (two threads per query row = TMEM lane, one per
+//     64-column half, in warps i and i + 4 of the tile, exchanging row max and
+//     sum through shared memory behind a 64-thread barrier per warp pair);
+//     warp 16 allocates tensor memory and issues every MMA from one thread;
+//     warp 17 streams K/V through the ring by TMA and warp 18 loads the Q
+//     tiles, each as soon as its slot frees.
+//   * Items are dealt to a persistent grid of one CTA per SM, heaviest first.
+//     With a causal mask tile 0 of an item ends one key tile before tile 1;
+//     S_0 of the next item's first key tile is then issued at once, so tile
+//     0's softmax warps do not idle across the item boundary.  (Issuing the
+//     two tiles' MMAs independently -- polled, or from two threads -- was
+//     measured slower: the two softmaxes then overlap and contend for the
+//     same pipes, where the fixed order below keeps them alternating.)
 //   * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
 //     The softmax writes P (bf16 pairs) over the first 64 columns of its S
 //     tile, and O += P V reads P straight from tensor memory (A operand in
@@ -32,7 +42,11 @@
 //   * Lazy rescale: the running max m moves (and O, l are rescaled) only
 //     when the new row max exceeds it by more than 2^8 in exp2 units; P is
 //     then at most 256, exact in the final O / l.
-//   * exp2 with scale*log2(e) folded into one FFMA per score.
+//   * exp2 with scale*log2(e) folded into one packed (f32x2) FMA per score
+//     pair.  One pair in eight takes 2^x from a cubic on the FMA pipe instead
+//     of the special-function unit, whose rate (16 results per clock per SM)
+//     otherwise equals the MMA rate for d = 128; more than that loads the FMA
+//     and issue slots more than it relieves the ex2 unit (measured).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -46,11 +60,13 @@ constexpr int D = 128;                  // head dimension
 constexpr int NS = 4;                   // K/V ring stages (K and V tiles interleaved)
 constexpr int TILE_BYTES = BM * D * 2;  // one 128 x 128 bf16 tile = 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;  // one 64-column half (a 128-byte-swizzled box)
-constexpr int NUM_THREADS = 576;     // 16 softmax warps + MMA warp + TMA warp
+constexpr int NUM_THREADS = 608;     // 16 softmax warps + MMA warp + K/V TMA warp + Q TMA warp
 constexpr int WG_THREADS = 256;      // one softmax warpgroup pair per query tile
 constexpr int MMA_WARP = 16;
-constexpr int TMA_WARP = 17;
+constexpr int TMA_WARP = 17;         // K/V stream
+constexpr int QLD_WARP = 18;         // Q tiles: loaded as soon as their slot frees
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPolyPairs = 1;  // of every 8 score pairs, those exponentiated on the FMA pipe
 
 struct Smem {
   // 1024-byte aligned by construction (the dynamic buffer is aligned at runtime).
@@ -92,27 +108,40 @@ __device__ __forceinline__ bool tile_needs_mask(int j, int r0, int n, int causal
   return (k1 >= n) || (causal && k1 > r0) || (window > 0 && k0 <= rlast - window);
 }
 
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+// 128-byte-swizzled shared-memory matrix descriptor as two 32-bit words: the
+// start address field (address >> 4, 14 bits) and the leading-byte offset in
+// the low word, stride offset, version and swizzle mode in the high word.  Shared
+// addresses stay below 2^18, so stepping through a tile is one add on the low
+// word with no carry out of the address field.
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) { return (saddr >> 4) | ((lbo >> 4) << 16); }
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo) { return (sbo >> 4) | (1u << 14) | (2u << 29); }
+__device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// S = Q K^T: Q and K tiles K-major ([64-column half][128 rows][64 cols]); a K step
+// of 16 columns is 32 bytes inside a half, the second half 16 KiB further on.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
   constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+  constexpr uint32_t hi = desc_hi(1024);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-    const uint64_t a = smem_desc_sw128(q_smem + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_smem + off, 16, 1024);
-    mma_ss(d_tmem, a, b, idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+    mma_ss(d_tmem, desc_of(q_lo + off, hi), desc_of(k_lo + off, hi), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem,
-                                         bool accumulate) {
+// O += P V: V tile MN-major ([64-column half][128 keys][64 cols]); a K step of 16
+// keys is 16 rows = 2 KiB.  P of keys [64h, 64h + 64) sits in S columns
+// [64h, 64h + 32) (bf16 pairs).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+  constexpr uint32_t hi = desc_hi(1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    // V tile: [64-column half][128 keys][64 cols]; a K step of 16 keys = 16 rows.
-    // P of keys [64h, 64h + 64) sits in S columns [64h, 64h + 32) (bf16 pairs).
-    const uint64_t b = smem_desc_sw128(v_smem + kk * 16 * 128, HALF_BYTES, 1024);
     const uint32_t a_col = (kk >> 2) * 64 + (kk & 3) * 8;
-    mma_ts(d_tmem, p_tmem + a_col, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d_tmem, p_tmem + a_col, desc_of(v_lo + ((kk * 16 * 128) >> 4), hi), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -201,18 +230,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == TMA_WARP) {
-    // ------------------------------------------------------------ producer
+  if (warp == QLD_WARP) {
+    // ------------------------------------------------------------ Q loader
+    // A warp of its own, so the next item's Q tile goes out as soon as the last
+    // S MMA of the current item has read the slot, ahead of the K/V stream.
     if (lane == 0) {
       int nq[2] = {0, 0};  // Q tiles loaded so far, per slot
-      int kvi = 0;         // K/V ring fills so far (K and V interleaved)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int lin = item_of(k, total);
         if (lin < 0) break;
         const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
         for (int t = 0; t < (it.has1 ? 2 : 1) && ok; ++t) {
-          // The slot is free once the previous item's last S_t MMA has completed.
           if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
           if (!ok) break;
           const uint32_t bar = smem_u32(&sm.q_full[t]);
@@ -221,6 +250,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, it.r0[t], it.bh);
           ++nq[t];
         }
+      }
+      for (int t = 0; t < 2; ++t)
+        if (nq[t] > 0) mbar_wait_drain(smem_u32(&sm.q_full[t]), (nq[t] - 1) & 1);
+    }
+  } else if (warp == TMA_WARP) {
+    // ------------------------------------------------------------ K/V producer
+    if (lane == 0) {
+      int kvi = 0;         // K/V ring fills so far (K and V interleaved)
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int lin = item_of(k, total);
+        if (lin < 0) break;
+        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
         for (int idx = 0; ok && idx < 2 * (it.hi - it.lo); ++idx, ++kvi) {
           const int s = kvi % NS;
           if (kvi >= NS) ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((kvi / NS) - 1) & 1, abort_flag);
@@ -235,33 +277,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // Drain: every copy issued must land before the CTA may exit.
       for (int i = max(0, kvi - NS); i < kvi; ++i) mbar_wait_drain(smem_u32(&sm.kv_full[i % NS]), (i / NS) & 1);
-      for (int t = 0; t < 2; ++t)
-        if (nq[t] > 0) mbar_wait_drain(smem_u32(&sm.q_full[t]), (nq[t] - 1) & 1);
     }
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t tS[2] = {tmem + 0, tmem + 128};
       const uint32_t tO[2] = {tmem + 256, tmem + 384};
-      const uint32_t q_s[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      // Descriptor low words of the Q slots (K-major, leading-byte offset 16).
+      const uint32_t q_s[2] = {desc_lo(smem_u32(sm.q[0]), 16), desc_lo(smem_u32(sm.q[1]), 16)};
       int nq[2] = {0, 0};    // Q tiles consumed, per slot
+      bool q_ready[2] = {false, false};  // slot t holds the tile now in use and was waited for
       int npv[2] = {0, 0};   // PV MMAs issued, per tile slot (p_full phase)
-      int nout[2] = {0, 0};  // items finished, per tile slot (o_free phase)
+      int nout[2] = {0, 0};  // items finished, per tile slot (o_full / o_free phase)
       int kvi = 0;
       bool ok = true;
+      bool s0_ahead = false;  // S_0(lo) of this item was issued during the previous item
       auto stage_of = [&](int i) { return i % NS; };
       auto parity_of = [&](int i) { return static_cast<uint32_t>((i / NS) & 1); };
+      // S_t(j) of item `it`: waits for the item's Q tile on first use; the item's last
+      // S_t releases the Q slot to the loader.
+      auto issue_s = [&](const Item& it, int t, int j, uint32_t ks) -> bool {
+        if (!q_ready[t]) {
+          if (!mbar_wait(smem_u32(&sm.q_full[t]), nq[t] & 1, abort_flag)) return false;
+          ++nq[t];
+          q_ready[t] = true;
+          tc_fence_after();
+        }
+        issue_qk(tS[t], q_s[t], ks);
+        tc_commit(smem_u32(&sm.s_full[t]));
+        if (j == it.hi_t[t] - 1) {
+          tc_commit(smem_u32(&sm.q_empty[t]));
+          q_ready[t] = false;
+        }
+        return true;
+      };
       for (int k = 0; ok; ++k) {
         const int lin = item_of(k, total);
         if (lin < 0) break;
         const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
         auto act = [&](int t, int j) { return j >= it.lo_t[t] && j < it.hi_t[t]; };
-        // S_t(j) and its bookkeeping: the last S_t of the item frees the Q slot.
-        auto issue_s = [&](int t, int j, uint32_t ks) {
-          issue_qk(tS[t], q_s[t], ks);
-          tc_commit(smem_u32(&sm.s_full[t]));
-          if (j == it.hi_t[t] - 1) tc_commit(smem_u32(&sm.q_empty[t]));
-        };
         // PV_t(j): the first one of an item overwrites O_t, so the previous item's
         // epilogue must have read it out; the last one publishes O_t.
         auto issue_o = [&](int t, int j, uint32_t vs) -> bool {
@@ -278,21 +332,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           return true;
         };
-        for (int t = 0; t < (it.has1 ? 2 : 1) && ok; ++t) {
-          ok = mbar_wait(smem_u32(&sm.q_full[t]), nq[t] & 1, abort_flag);
-          ++nq[t];
-        }
-        if (!ok || it.hi <= it.lo) break;
-        // Prologue: S_t(lo) for both tiles.
+        if (it.hi <= it.lo) break;
+        // Prologue: S_t(lo) for both tiles (S_0(lo) may already be in flight).
         ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi)]), parity_of(kvi), abort_flag);
         if (!ok) break;
         tc_fence_after();
         {
-          const uint32_t ks = smem_u32(sm.kv[stage_of(kvi)]);
-          for (int t = 0; t < 2; ++t)
-            if (act(t, it.lo)) issue_s(t, it.lo, ks);
+          const uint32_t ks = desc_lo(smem_u32(sm.kv[stage_of(kvi)]), 16);
+          for (int t = 0; t < 2 && ok; ++t)
+            if (act(t, it.lo) && !(t == 0 && s0_ahead)) ok = issue_s(it, t, it.lo, ks);
+          if (!ok) break;
           tc_commit(smem_u32(&sm.kv_empty[stage_of(kvi)]));
           ++kvi;
+          s0_ahead = false;
         }
         for (int j = it.lo; ok && j < it.hi; ++j) {
           const int vidx = kvi;            // V_j
@@ -301,23 +353,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(vidx)]), parity_of(vidx), abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vs = smem_u32(sm.kv[stage_of(vidx)]);
+          const uint32_t vs = desc_lo(smem_u32(sm.kv[stage_of(vidx)]), HALF_BYTES);
           if (act(0, j) && !(ok = issue_o(0, j, vs))) break;
           uint32_t ks = 0;
           if (has_next) {
             ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(nidx)]), parity_of(nidx), abort_flag);
             if (!ok) break;
             tc_fence_after();
-            ks = smem_u32(sm.kv[stage_of(nidx)]);
-            if (act(0, j + 1)) issue_s(0, j + 1, ks);
+            ks = desc_lo(smem_u32(sm.kv[stage_of(nidx)]), 16);
+            if (act(0, j + 1) && !(ok = issue_s(it, 0, j + 1, ks))) break;
           }
           if (act(1, j) && !(ok = issue_o(1, j, vs))) break;
           tc_commit(smem_u32(&sm.kv_empty[stage_of(vidx)]));
           if (has_next) {
-            if (act(1, j + 1)) issue_s(1, j + 1, ks);
+            if (act(1, j + 1) && !(ok = issue_s(it, 1, j + 1, ks))) break;
             tc_commit(smem_u32(&sm.kv_empty[stage_of(nidx)]));
           }
           kvi += has_next ? 2 : 1;
+          // Causal masks end tile 0 one key tile before tile 1.  Its softmax warps
+          // would then idle until tile 1 finishes, so S_0 of the next item's first
+          // key tile goes out now: K(lo') is the ring entry after V(hi - 1), and
+          // ring entry kvi + 1 - NS has been consumed already.
+          if (j == it.hi - 2 && it.has1 && !act(0, j + 1)) {
+            const int lin2 = item_of(k + 1, total);
+            if (lin2 >= 0) {
+              const Item nx = make_item(lin2, BH, n, num_pairs, args.causal, args.window);
+              if (nx.hi > nx.lo && nx.lo_t[0] == nx.lo) {
+                ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi + 1)]), parity_of(kvi + 1), abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                if (!(ok = issue_s(nx, 0, nx.lo, desc_lo(smem_u32(sm.kv[stage_of(kvi + 1)]), 16)))) break;
+                s0_ahead = true;
+              }
+            }
+          }
         }
       }
       // All MMAs issued by this thread must complete before TMEM is freed.
@@ -334,7 +403,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int wi = warp & 7;
     const int hc = wi >> 2;          // column half
     const int row = (wi & 3) * 32 + lane;
-    const int bar_id = 1 + t;        // named barrier of this tile's 256 threads
+    // The two threads of a row sit in warps wi and wi + 4 (same TMEM lanes); only
+    // that warp pair exchanges, on a 64-thread named barrier of its own.
+    const int bar_id = 3 + 4 * t + (wi & 3);
+    constexpr int kBarThreads = 64;
     const uint32_t lane_off = static_cast<uint32_t>((wi & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128 + 64 * hc;
     const uint32_t tO = tmem + lane_off + 256 + t * 128 + 64 * hc;
@@ -385,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sm.xmax[t][ns & 1][hc][row] = hm;
         // Barrier of the tile's 256 threads: both halves' maxima are visible, and the
         // whole group agrees on whether to go on.
-        ok = named_bar_all(ok, bar_id, WG_THREADS);
+        ok = named_bar_all(ok, bar_id, kBarThreads);
         if (!ok) break;
         const float mx = fmax3_nan(hm, sm.xmax[t][ns & 1][hc ^ 1][row], -INFINITY);
         nan_row |= (mx != mx);
@@ -402,22 +474,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         const float ms = (m == -INFINITY) ? 0.f : m * sl2;
         // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> bf16 pairs over this
-        // half's first 32 S columns (already read).
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+        // half's first 32 S columns (already read).  Scores go in pairs through the
+        // packed f32x2 FMA; kPolyPairs of every 8 pairs take 2^x from the cubic on
+        // the FMA pipe, the rest from the special-function unit, so both pipes share
+        // the exponentials.
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nms2 = f2_pack(-ms, -ms);
+        uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t p[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(s[32 * c + e]), sl2, -ms));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(s[32 * c + e + 1]), sl2, -ms));
-            if (e & 2) {
-              acc2 += p0;
-              acc3 += p1;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[32 * c + e]), __uint_as_float(s[32 * c + e + 1])),
+                                       sl2x2, nms2);
+            uint64_t p2;
+            if (((e >> 1) & 7) >= 8 - kPolyPairs) {
+              p2 = exp2_poly_pair(x2);
             } else {
-              acc0 += p0;
-              acc1 += p1;
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
             }
+            if (e & 2) acc_b = f2_add(acc_b, p2); else acc_a = f2_add(acc_a, p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
             p[e >> 1] = pack_bf16x2(p0, p1);
           }
           asm volatile(
@@ -442,7 +522,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sm.p_full[t]));
-        l += (acc0 + acc1) + (acc2 + acc3);
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(acc_a, a0, a1);
+          f2_unpack(acc_b, b0, b1);
+          l += (a0 + a1) + (b0 + b1);
+        }
       }
       if (!ok) break;
       // Epilogue: O / l in bf16 and lse = m * scale + ln l.  O_t is read out first and
@@ -456,7 +541,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       sm.xsum[t][hc][row] = l;
-      ok = named_bar_all(ok, bar_id, WG_THREADS);
+      ok = named_bar_all(ok, bar_id, kBarThreads);
       mbar_arrive(smem_u32(&sm.o_free[t]));
       if (!ok) break;
       float lt = l + sm.xsum[t][hc ^ 1][row];
