@@ -353,7 +353,10 @@ def run_gpu(args, rank, world, local_rank):
     roof["traffic"] = profiled_traffic(kernel, w.name, sources)
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms,
+        "ms_per_step_spread": {"p50": float(np.median(times)), "min": float(np.min(times)),
+                               "max": float(np.max(times))},
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), workloads.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "window": w.window, "global_batch": w.B * world, "seq_len": w.N,
