@@ -32,6 +32,19 @@ def test_bf16_forward_small(N, causal, window):
     assert_lse_close(lse, lse_ref, f"lse N={N} causal={causal} window={window}")
 
 
+@pytest.mark.parametrize("causal,window", [(True, 0), (True, 200), (False, 0), (False, 300)])
+def test_bf16_forward_many_items_per_cta(causal, window):
+    """160 heads x 3 row pairs = 480 work items for at most 148 persistent CTAs, so
+    every CTA walks several items and crosses item boundaries (where the next
+    item's first S may be issued early); N = 640 leaves the last pair with a single
+    query tile."""
+    q, k, v = workloads.forward_inputs(4, 40, 640, 128, torch.bfloat16, seed=31 + window, device="cpu")
+    o, lse = run_fwd(q.cuda(), k.cuda(), v.cuda(), causal, window)
+    O_ref, lse_ref = oracle.attention_forward(q, k, v, None, causal, window)
+    assert_output_close(o, O_ref, f"O many items causal={causal} window={window}")
+    assert_lse_close(lse, lse_ref, f"lse many items causal={causal} window={window}")
+
+
 def test_bf16_forward_explicit_scale_and_no_lse():
     q, k, v = workloads.forward_inputs(1, 2, 200, 128, torch.bfloat16, seed=11, device="cuda")
     o = torch.empty_like(q)

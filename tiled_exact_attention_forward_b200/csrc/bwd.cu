@@ -57,7 +57,6 @@ struct Smem {
   uint64_t qdo_full[2];
   uint64_t qdo_empty[2];
   uint64_t s_full, dp_full, ds_ready, dq_full, dq_free, acc_done;
-  uint64_t stage_free;  // dQ staging (in the dS buffer) read by the TMA (dQ group -> P/dS group)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -143,7 +142,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&sm.kv_full), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&sm.qdo_full[s]), 1);
-      mbar_init(smem_u32(&sm.qdo_empty[s]), 1);
+      // Two arrivals free a (Q, dO) slot: the MMAs that read it, and the TMA reduce
+      // that read the dQ staged in it afterwards.
+      mbar_init(smem_u32(&sm.qdo_empty[s]), 2);
     }
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.dp_full), 1);
@@ -151,7 +152,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&sm.dq_full), 1);
     mbar_init(smem_u32(&sm.dq_free), GROUP);
     mbar_init(smem_u32(&sm.acc_done), 1);
-    mbar_init(smem_u32(&sm.stage_free), 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -327,9 +327,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7])
                      : "memory");
         // dS (queries 64h + 16c .. +15 of this key row) into the swizzled MN-major tile.
-        // The buffer doubles as the previous step's dQ staging: wait until the TMA has
-        // read that out (usually long done).
-        if (c == 0 && idx > 0) ok = mbar_wait_warp(smem_u32(&sm.stage_free), (idx - 1) & 1, abort_flag) && ok;
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int chunk = (c * 2 + u) ^ (row & 7);
@@ -386,34 +383,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.dq_free));  // TMEM read: the next S^T may overwrite it
-      // Stage through the 32 KiB dS buffer in two rounds (column half 0, then 1):
-      // two 32-column x 128-row float boxes, 128-byte swizzled, reduced into the
-      // fp32 accumulator by the TMA (rows past N are skipped by the TMA).
-      for (int round = 0; round < 2; ++round) {
-        if (hc == round && ok) {
+      // Stage in the (Q, dO) slot of this query tile -- its last readers, the dV and
+      // dK MMAs, completed before dQ -- as four 32-column x 128-row float boxes,
+      // 128-byte swizzled, reduced into the fp32 accumulator by the TMA (rows past N
+      // are skipped by the TMA).  The slot is handed back to the loader once the TMA
+      // has read the staging; it refills it two query tiles later.
+      const int s = idx & 1;
+      if (ok) {
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            uint8_t* box = sm.ds + b * (BQ * 128) + row * 128;
+        for (int b = 0; b < 2; ++b) {
+          uint8_t* box = (hc == 0 ? sm.q[s] : sm.dout[s]) + b * (BQ * 128) + row * 128;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const int e = 32 * b + 4 * ch;
-              *reinterpret_cast<float4*>(box + ((ch ^ (row & 7)) * 16)) =
-                  make_float4(__uint_as_float(r[e]) * scale, __uint_as_float(r[e + 1]) * scale,
-                              __uint_as_float(r[e + 2]) * scale, __uint_as_float(r[e + 3]) * scale);
-            }
+          for (int ch = 0; ch < 8; ++ch) {
+            const int e = 32 * b + 4 * ch;
+            *reinterpret_cast<float4*>(box + ((ch ^ (row & 7)) * 16)) =
+                make_float4(__uint_as_float(r[e]) * scale, __uint_as_float(r[e + 1]) * scale,
+                            __uint_as_float(r[e + 2]) * scale, __uint_as_float(r[e + 3]) * scale);
           }
-          fence_proxy_async_smem();
         }
-        ok = named_bar_all(ok, 3, GROUP);
-        if (gt == 0 && ok) {
-          tma_reduce_add_3d(&tm_dq, smem_u32(sm.ds), 64 * round, q0, bh);
-          tma_reduce_add_3d(&tm_dq, smem_u32(sm.ds) + BQ * 128, 64 * round + 32, q0, bh);
-          bulk_commit();
-          bulk_wait_read0();  // the staging may be rewritten once the TMA has read it
-        }
-        ok = named_bar_all(ok, 3, GROUP);
+        fence_proxy_async_smem();
       }
-      if (gt == 0) mbar_arrive(smem_u32(&sm.stage_free));
+      ok = named_bar_all(ok, 3, GROUP);
+      if (gt == 0) {
+        if (ok) {
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.q[s]), 0, q0, bh);
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.q[s]) + BQ * 128, 32, q0, bh);
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.dout[s]), 64, q0, bh);
+          tma_reduce_add_3d(&tm_dq, smem_u32(sm.dout[s]) + BQ * 128, 96, q0, bh);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        mbar_arrive(smem_u32(&sm.qdo_empty[s]));
+      }
       if (!ok) break;
     }
     if (gt == 0) bulk_wait0();  // every reduce-add has landed before the CTA ends
