@@ -79,12 +79,6 @@ __device__ __forceinline__ bool tile_needs_mask(int kt, int qi, int n, int causa
   return (k1 >= n) || (causal && q0 < k1) || (window > 0 && q1 - k0 >= window);
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
 // A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
 __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
@@ -96,14 +90,17 @@ __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint
   }
 }
 
-// D[128 x d] (+)= A[tmem, 128 x 128 bf16] * B, B = [128 rows (K)][d] tile (MN-major).
-// A's K columns [64h, 64h + 64) (bf16 pairs) sit at TMEM columns [64h, 64h + 32).
-__device__ __forceinline__ void issue_tmemA_b(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
-                                              bool accumulate) {
+// D[128 x d] (+)= A[tmem, 128 keys x 64 queries of half H, bf16] * B, B = [128 rows (K)][d]
+// tile (MN-major), rows 64H .. 64H + 63.  The A columns of queries [16k, 16k + 16) sit at
+// TMEM columns 64 (k / 4) + 32 ((k % 4) / 2) + 8 (k % 2) (bf16 pairs), where the P/dS
+// thread that owns those queries wrote them over S^T / dP^T columns it had read.
+template <int H>
+__device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
+                                                   bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8,
+  for (int kk = 4 * H; kk < 4 * H + 4; ++kk)
+    mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8,
            smem_desc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -205,11 +202,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int idx = 0; ok && idx < nq; ++idx) {
         const int s = idx & 1;
-        ok = mbar_wait(smem_u32(&sm.ds_ready), idx & 1, abort_flag);
+        // dV and dK for query half 0 as soon as its P^T and dS^T are in TMEM (they run
+        // while the P/dS warps work on half 1), then half 1 (two ds_ready phases per
+        // query tile: parity 0, then 1).
+        ok = mbar_wait(smem_u32(&sm.ds_ready), 0, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_tmemA_b(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
-        issue_tmemA_b(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
+        issue_tmemA_b_half<0>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
+        issue_tmemA_b_half<0>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
+        ok = mbar_wait(smem_u32(&sm.ds_ready), 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        issue_tmemA_b_half<1>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), true);
+        issue_tmemA_b_half<1>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), true);
         tc_commit(smem_u32(&sm.qdo_empty[s]));
         issue_dq(tmem + T_S, dss, ks);
         tc_commit(smem_u32(&sm.dq_full));
@@ -232,16 +237,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     __syncwarp();
   } else if (warp < 8) {
-    // -------------------------------------------------- P^T and dS^T (thread = key row x 64 queries)
-    const int hc = warp >> 2;
+    // -------------------------------------------------- P^T and dS^T (thread = key row x 32 queries
+    // of each query half, the halves one after the other)
+    const int hc = warp >> 2;  // which 32 queries of a half (and, at the end, which dV columns)
     const int row = (warp & 3) * 32 + lane;
     const int key = kt * BM + row;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + T_S + 64 * hc, tDP = tmem + lane_off + T_DP + 64 * hc;
+    const uint32_t tSb = tmem + lane_off + T_S + 32 * hc, tDPb = tmem + lane_off + T_DP + 32 * hc;
     const float sl2 = args.scale_log2;
     const float* lse_g = args.lse + static_cast<size_t>(bh) * n;
     const float* del_g = args.ws_delta + static_cast<size_t>(bh) * n;
-    uint8_t* ds_row = sm.ds + hc * HALF_BYTES + row * 128;
     const int gt = threadIdx.x;  // 0..255: loads row statistic gt & 127 (lse if < 128, else D)
     bool ok = true;
     // Prefetch the first tile's row statistics.
@@ -272,72 +277,78 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = named_bar_all(ok, 2, GROUP);
       if (!ok) break;
       tc_fence_after();
-      // Visible queries of this key row form one interval [q_lo, q_hi) of this half.
-      int q_lo = 0, q_hi = 64;
-      if (masked) {
-        const int qbase = qt * BQ + 64 * hc;
-        if (args.causal) q_lo = max(0, key - qbase);
-        if (args.window > 0) q_hi = min(64, key + args.window - qbase);
-        q_hi = min(q_hi, n - qbase);  // queries past N have lse2 = +inf anyway
-        if (key >= n) q_hi = 0;
-      }
-      const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][64 * hc]);
-      const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[s][64 * hc]);
-      // 16 query columns per step keeps S^T, dP^T and both outputs in registers.
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t tS = tSb + 64 * h, tDP = tDPb + 64 * h;
+        // Visible queries of this key row form one interval [q_lo, q_hi) of its 32.
+        int q_lo = 0, q_hi = 32;
+        if (masked) {
+          const int qbase = qt * BQ + 64 * h + 32 * hc;
+          if (args.causal) q_lo = max(0, key - qbase);
+          if (args.window > 0) q_hi = min(32, key + args.window - qbase);
+          q_hi = min(q_hi, n - qbase);  // queries past N have lse2 = +inf anyway
+          if (key >= n) q_hi = 0;
+        }
+        const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][64 * h + 32 * hc]);
+        const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[s][64 * h + 32 * hc]);
+        uint8_t* ds_row = sm.ds + h * HALF_BYTES + row * 128;
+        // 16 query columns per step keeps S^T, dP^T and both outputs in registers.
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sr[16], dr[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(sr[0]), "=r"(sr[1]), "=r"(sr[2]), "=r"(sr[3]), "=r"(sr[4]), "=r"(sr[5]), "=r"(sr[6]), "=r"(sr[7]),
-              "=r"(sr[8]), "=r"(sr[9]), "=r"(sr[10]), "=r"(sr[11]), "=r"(sr[12]), "=r"(sr[13]), "=r"(sr[14]), "=r"(sr[15])
-            : "r"(tS + 16 * c));
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(dr[0]), "=r"(dr[1]), "=r"(dr[2]), "=r"(dr[3]), "=r"(dr[4]), "=r"(dr[5]), "=r"(dr[6]), "=r"(dr[7]),
-              "=r"(dr[8]), "=r"(dr[9]), "=r"(dr[10]), "=r"(dr[11]), "=r"(dr[12]), "=r"(dr[13]), "=r"(dr[14]), "=r"(dr[15])
-            : "r"(tDP + 16 * c));
-        tmem_ld_wait();
-        uint32_t pp[8], dd[8];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sr[16], dr[16];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+              : "=r"(sr[0]), "=r"(sr[1]), "=r"(sr[2]), "=r"(sr[3]), "=r"(sr[4]), "=r"(sr[5]), "=r"(sr[6]), "=r"(sr[7]),
+                "=r"(sr[8]), "=r"(sr[9]), "=r"(sr[10]), "=r"(sr[11]), "=r"(sr[12]), "=r"(sr[13]), "=r"(sr[14]), "=r"(sr[15])
+              : "r"(tS + 16 * c));
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+              : "=r"(dr[0]), "=r"(dr[1]), "=r"(dr[2]), "=r"(dr[3]), "=r"(dr[4]), "=r"(dr[5]), "=r"(dr[6]), "=r"(dr[7]),
+                "=r"(dr[8]), "=r"(dr[9]), "=r"(dr[10]), "=r"(dr[11]), "=r"(dr[12]), "=r"(dr[13]), "=r"(dr[14]), "=r"(dr[15])
+              : "r"(tDP + 16 * c));
+          tmem_ld_wait();
+          uint32_t pp[8], dd[8];
 #pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4) {
-          const float4 lv = l4[4 * c + e4];
-          const float4 dv = d4[4 * c + e4];
-          const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-          const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
-          float pv[4], dsv[4];
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 lv = l4[4 * c + e4];
+            const float4 dv = d4[4 * c + e4];
+            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+            const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+            float pv[4], dsv[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int e = 4 * e4 + u;
-            float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lq[u]));
-            if (masked && (16 * c + e < q_lo || 16 * c + e >= q_hi)) p = 0.f;
-            pv[u] = p;
-            dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
+            for (int u = 0; u < 4; ++u) {
+              const int e = 4 * e4 + u;
+              float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lq[u]));
+              if (masked && (16 * c + e < q_lo || 16 * c + e >= q_hi)) p = 0.f;
+              pv[u] = p;
+              dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
+            }
+            pp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
+            pp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
+            dd[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
+            dd[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          pp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
-          pp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dd[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
-          dd[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-        }
-        // P^T over S^T columns [64h + 8c, +8), dS^T over dP^T columns (both already read).
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tS + 8 * c),
-                     "r"(pp[0]), "r"(pp[1]), "r"(pp[2]), "r"(pp[3]), "r"(pp[4]), "r"(pp[5]), "r"(pp[6]), "r"(pp[7])
-                     : "memory");
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tDP + 8 * c),
-                     "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7])
-                     : "memory");
-        // dS (queries 64h + 16c .. +15 of this key row) into the swizzled MN-major tile.
+          // P^T over this thread's S^T columns [8c, 8c + 8) (already read), dS^T likewise
+          // over its dP^T columns.
+          asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tS + 8 * c),
+                       "r"(pp[0]), "r"(pp[1]), "r"(pp[2]), "r"(pp[3]), "r"(pp[4]), "r"(pp[5]), "r"(pp[6]), "r"(pp[7])
+                       : "memory");
+          asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(tDP + 8 * c),
+                       "r"(dd[0]), "r"(dd[1]), "r"(dd[2]), "r"(dd[3]), "r"(dd[4]), "r"(dd[5]), "r"(dd[6]), "r"(dd[7])
+                       : "memory");
+          // dS (queries 64h + 32hc + 16c .. +15 of this key row) into the swizzled
+          // MN-major tile.
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int chunk = (c * 2 + u) ^ (row & 7);
-          *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
-              make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+          for (int u = 0; u < 2; ++u) {
+            const int chunk = (4 * hc + 2 * c + u) ^ (row & 7);
+            *reinterpret_cast<uint4*>(ds_row + chunk * 16) =
+                make_uint4(dd[4 * u], dd[4 * u + 1], dd[4 * u + 2], dd[4 * u + 3]);
+          }
         }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.ds_ready));
       }
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&sm.ds_ready));
     }
     // Epilogue: dV rows (64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
