@@ -106,3 +106,21 @@ def test_python_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.forward(q, q, q)
+
+
+def test_forward_host_checks_its_inputs_before_touching_the_device():
+    import torch
+
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward_host(q.transpose(2, 3), q, q)  # not contiguous
+    with pytest.raises(ValueError):
+        fa.forward_host(q, q[:, :1], q)  # shapes differ
+
+
+def test_forward_backward_host_checks_its_inputs():
+    import torch
+
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward_backward_host(q, q, q, q.float())  # dout dtype differs

@@ -45,6 +45,20 @@ def test_bf16_forward_many_items_per_cta(causal, window):
     assert_lse_close(lse, lse_ref, f"lse many items causal={causal} window={window}")
 
 
+@pytest.mark.parametrize("chunks", [1, 4, 6, 100])
+def test_forward_host_pipelined_over_head_groups(chunks):
+    """forward_host splits the 2 x 3 heads into `chunks` groups (clamped to 6) whose
+    copies and kernels overlap on three streams; results equal the oracle's."""
+    q, k, v = workloads.forward_inputs(2, 3, 300, 128, torch.bfloat16, seed=41, device="cpu")
+    q, k, v = (t.pin_memory() for t in (q, k, v))
+    o, lse = fa.forward_host(q, k, v, causal=True, window=100, chunks=chunks)
+    assert not o.is_cuda and o.shape == q.shape and lse.shape == (2, 3, 300)
+    assert fa.device_status() == fa.FA_OK
+    O_ref, lse_ref = oracle.attention_forward(q, k, v, None, True, 100)
+    assert_output_close(o, O_ref, f"forward_host O chunks={chunks}")
+    assert_lse_close(lse, lse_ref, f"forward_host lse chunks={chunks}")
+
+
 def test_bf16_forward_explicit_scale_and_no_lse():
     q, k, v = workloads.forward_inputs(1, 2, 200, 128, torch.bfloat16, seed=11, device="cuda")
     o = torch.empty_like(q)

@@ -12,6 +12,7 @@ Functions (names follow the C ABI):
     backward(q, k, v, o, dout, lse, causal=False, window=0,
              scale=None)                                         -> (dq, dk, dv)
     forward_host(...)  -- forward on pinned host tensors (copies in and out)
+    forward_backward_host(...)  -- forward and backward on pinned host tensors
     device_status()    -- FA_OK or the first recorded device-side timeout
 """
 from __future__ import annotations
@@ -145,20 +146,108 @@ def forward(q, k, v, causal: bool = False, window: int = 0, scale=None, out=None
     return o, lse
 
 
-def forward_host(q, k, v, causal: bool = False, window: int = 0, scale=None, device="cuda"):
-    """The forward for host tensors: copy in (pinned -> device), run, copy out.
+_HOST_STREAMS = {}
 
-    Returns host (o, lse).  The copies are ordered on the current stream.
+
+def _host_streams(dev):
+    """Three side streams per device (copy in, compute, copy out), made once."""
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _HOST_STREAMS:
+        _HOST_STREAMS[key] = tuple(torch.cuda.Stream(device=dev) for _ in range(3))
+    return _HOST_STREAMS[key]
+
+
+def _host_pipelined(dev, host_ins, out_specs, chunks, compute):
+    """Runs `compute` over head groups with the copies pipelined around it.
+
+    host_ins: host tensors whose first dimension is the B * H heads; out_specs:
+    (trailing shape, dtype) of each output, also head-major.  For each group of
+    heads [a, b): the inputs are copied in on one stream, compute(a, b, dev_ins,
+    dev_outs) runs on a second, the outputs are copied back on a third, so the
+    copy-in of one group overlaps the kernels of the previous group and the
+    copy-out of the one before (PCIe moves both directions at once).  The
+    copy-in stream first waits for the work already queued on the current
+    stream; the call returns once the results are in (pinned) host memory.
     """
+    BH = host_ins[0].shape[0]
+    chunks = max(1, min(int(chunks), BH))
+    dev_ins = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in host_ins]
+    dev_outs = [torch.empty((BH, *tail), dtype=dt, device=dev) for tail, dt in out_specs]
+    host_outs = [torch.empty((BH, *tail), dtype=dt, pin_memory=True) for tail, dt in out_specs]
+    s_in, s_run, s_out = _host_streams(dev)
+    cur = torch.cuda.current_stream(dev)
+    s_in.wait_stream(cur)
+    bounds = [(g * BH) // chunks for g in range(chunks + 1)]
+    for g in range(chunks):
+        a, b = bounds[g], bounds[g + 1]
+        with torch.cuda.stream(s_in):
+            for dst, src in zip(dev_ins, host_ins):
+                dst[a:b].copy_(src[a:b], non_blocking=True)
+        s_run.wait_stream(s_in)
+        with torch.cuda.stream(s_run):
+            compute(a, b, dev_ins, dev_outs)
+        s_out.wait_stream(s_run)
+        with torch.cuda.stream(s_out):
+            for dst, src in zip(host_outs, dev_outs):
+                dst[a:b].copy_(src[a:b], non_blocking=True)
+    cur.wait_stream(s_out)
+    s_out.synchronize()
+    return host_outs, max(bounds[g + 1] - bounds[g] for g in range(chunks))
+
+
+def _check_host(*ts):
+    for t in ts:
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host-buffer calls take contiguous host tensors")
+    if any(t.shape != ts[0].shape or t.dtype != ts[0].dtype for t in ts):
+        raise ValueError("q, k, v (and dout) must share shape and dtype")
+
+
+def forward_host(q, k, v, causal: bool = False, window: int = 0, scale=None, device="cuda", chunks: int = 4):
+    """The forward for host tensors: copy in, run, copy out; returns pinned host (o, lse).
+
+    q, k, v: contiguous [B, H, N, d] host tensors (pinned memory makes the copies
+    asynchronous).  Every (batch, head) is independent, so the heads go through
+    in `chunks` groups with copies and kernels overlapped (see _host_pipelined).
+    """
+    _check_host(q, k, v)
     dev = torch.device(device)
-    qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    o, lse = forward(qd, kd, vd, causal, window, scale)
-    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    o_h.copy_(o, non_blocking=True)
-    l_h.copy_(lse, non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
-    return o_h, l_h
+    B, H, N, d = q.shape
+
+    def run(a, b, ins, outs):
+        qd, kd, vd = (t[a:b].unsqueeze(0) for t in ins)
+        forward(qd, kd, vd, causal, window, scale, out=outs[0][a:b].unsqueeze(0), lse=outs[1][a:b].unsqueeze(0))
+
+    (o, lse), _ = _host_pipelined(dev, [t.reshape(B * H, N, d) for t in (q, k, v)],
+                                  [((N, d), q.dtype), ((N,), torch.float32)], chunks, run)
+    return o.view(B, H, N, d), lse.view(B, H, N)
+
+
+def forward_backward_host(q, k, v, dout, causal: bool = False, window: int = 0, scale=None, device="cuda",
+                          chunks: int = 8):
+    """Forward and backward for host tensors; returns pinned host (o, lse, dq, dk, dv).
+
+    The heads go through in `chunks` groups with copies and kernels overlapped
+    (see _host_pipelined); the backward's workspace is sized for the largest
+    group and reused, the groups' kernels running in order on one stream.
+    """
+    _check_host(q, k, v, dout)
+    dev = torch.device(device)
+    B, H, N, d = q.shape
+    chunks = max(1, min(int(chunks), B * H))
+    largest = -(-(B * H) // chunks)
+    ws = torch.empty(max(backward_workspace_size(1, largest, N, d), 256), dtype=torch.uint8, device=dev)
+
+    def run(a, b, ins, outs):
+        qd, kd, vd, gd = (t[a:b].unsqueeze(0) for t in ins)
+        od, ld, dqd, dkd, dvd = (t[a:b].unsqueeze(0) for t in outs)
+        forward(qd, kd, vd, causal, window, scale, out=od, lse=ld)
+        backward(qd, kd, vd, od, gd, ld, causal, window, scale, workspace=ws, dq=dqd, dk=dkd, dv=dvd)
+
+    specs = [((N, d), q.dtype), ((N,), torch.float32)] + [((N, d), q.dtype)] * 3
+    outs, _ = _host_pipelined(dev, [t.reshape(B * H, N, d) for t in (q, k, v, dout)], specs, chunks, run)
+    o, lse, dq, dk, dv = outs
+    return o.view(B, H, N, d), lse.view(B, H, N), dq.view(B, H, N, d), dk.view(B, H, N, d), dv.view(B, H, N, d)
 
 
 def decode_workspace_size(B, H, cap, d) -> int:
