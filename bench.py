@@ -6,12 +6,14 @@ One step is one pass of the hot path over one batch of synthetic input:
   causal_prefill (default): fa_forward on B=4, H=16, N=2048, d=128, bf16, causal
   sliding_window_long:      fa_forward on B=1, H=32, N=16384, d=128, window 4096
   kv_cache_decode:          fa_decode, batch 64 x 32 heads, cache lengths U[512, 8192]
+  paged_kv_decode:          fa_decode_paged, the same lengths in shuffled 16-row blocks of one pool
   causal_fwd_bwd:           fa_forward + fa_backward on B=2, H=16, N=4096, d=128
 Inputs are seeded N(0,1) draws (``workloads.py``), resident in HBM before the
 timed region.  The L2 (126 MB) is flushed between timed steps by writing a
 256 MiB buffer outside the timed events.  Throughput counts only the (query,
 key) pairs the mask allows: 4*d FLOPs per pair forward, 10*d backward;
-decode counts the bytes of the K/V rows it must read plus q and o.
+decode counts the bytes of the K/V rows it must read plus q and o (paged: plus
+the block-table entries it uses).
 
 Prints one JSON line (rank 0).  With --gpus N > 1 (launched by torchrun) each
 rank runs its own independent batch (weak scaling, no collective on the data
@@ -61,9 +63,14 @@ def backward_flops(w) -> float:
     return 10.0 * w.d * allowed_pairs(w.N, w.causal, w.window) * w.B * w.H
 
 
+DECODE_KINDS = ("decode", "paged_decode")
+
+
 def decode_bytes(w, seqlens) -> float:
-    rows = float(np.minimum(np.asarray(seqlens, dtype=np.int64), w.N).sum()) * w.H
-    return rows * w.d * 2 * 2 + 2 * w.B * w.H * w.d * 2  # K + V rows, q + o
+    n = np.minimum(np.asarray(seqlens, dtype=np.int64), w.N)
+    rows = float(n.sum()) * w.H
+    table = 4.0 * float((-(-n // w.block_size)).sum()) if w.kind == "paged_decode" else 0.0
+    return rows * w.d * 2 * 2 + 2 * w.B * w.H * w.d * 2 + table  # K + V rows, q + o, table
 
 
 # ----------------------------------------------------------------------------- measurement helpers
@@ -189,6 +196,17 @@ def oracle_sample(w, budget_s=12.0):
             oracle.decode_forward(q, kc, vc, np.array([n]), w.scale)
             t_total += time.perf_counter() - t0
             units += n * w.d * 2 * 2 + 2 * w.d * 2
+        elif w.kind == "paged_decode":
+            n = int(workloads.decode_seqlens(w.B, w.seqlen_lo, w.seqlen_hi, w.seed)[heads % w.B])
+            nb = -(-n // w.block_size)
+            q = torch.randn(1, 1, w.d, generator=gen).to(w.dtype)
+            kp = torch.randn(nb, 1, w.block_size, w.d, generator=gen).to(w.dtype)
+            vp = torch.randn(nb, 1, w.block_size, w.d, generator=gen).to(w.dtype)
+            table = torch.randperm(nb, generator=gen).reshape(1, nb)
+            t0 = time.perf_counter()
+            oracle.decode_paged_forward(q, kp, vp, table, np.array([n]), w.scale)
+            t_total += time.perf_counter() - t0
+            units += n * w.d * 2 * 2 + 2 * w.d * 2 + 4 * nb
         else:
             q, k, v = (torch.randn(w.N, w.d, generator=gen).to(w.dtype) for _ in range(3))
             t0 = time.perf_counter()
@@ -203,7 +221,7 @@ def oracle_sample(w, budget_s=12.0):
             units += per
         heads += 1
     rate = units / t_total
-    if w.kind == "decode":
+    if w.kind in DECODE_KINDS:
         return rate / 1e9, f"{heads} of {w.B * w.H} (sequence, head) decodes, {t_total:.1f} s"
     return rate / 1e12, f"{heads} of {w.B * w.H} heads (full N x N float64 per head), {t_total:.1f} s"
 
@@ -212,6 +230,35 @@ def oracle_sample(w, budget_s=12.0):
 def make_step(w, dev):
     """Returns (step_fn, e2e_fn, units_per_step, unit, metric, launches_per_step, kernel, sources)."""
     import tiled_exact_attention_forward_b200 as fa
+
+    if w.kind == "paged_decode":
+        q, kp, vp, table, seqlens = workloads.workload_inputs(w, device=dev)
+        ws = torch.empty(fa.decode_workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H), dtype=torch.float32, device=dev)
+        units = decode_bytes(w, seqlens.cpu().numpy()) / 1e9
+
+        def step():
+            fa.decode_paged(q, kp, vp, table, seqlens, w.scale, workspace=ws, out=o, lse=lse)
+
+        # End to end: the step's own inputs (new query, lengths, block table) go up and
+        # the output comes back; the block pool stays resident as it would in serving.
+        q_h, s_h, t_h = (t.cpu().pin_memory() for t in (q, seqlens, table))
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        l_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e():
+            q.copy_(q_h, non_blocking=True)
+            seqlens.copy_(s_h, non_blocking=True)
+            table.copy_(t_h, non_blocking=True)
+            fa.decode_paged(q, kp, vp, table, seqlens, w.scale, workspace=ws, out=o, lse=lse)
+            o_h.copy_(o, non_blocking=True)
+            l_h.copy_(lse, non_blocking=True)
+
+        h2d = sum(t.numel() * t.element_size() for t in (q_h, s_h, t_h))
+        d2h = o_h.numel() * o_h.element_size() + l_h.numel() * 4
+        return (step, e2e, units, "GB/s", "decode GB/s", 2, "decode_split_kernel",
+                ["decode.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
     if w.kind == "decode":
         q, kc, vc, seqlens = workloads.workload_inputs(w, device=dev)
@@ -363,7 +410,8 @@ def run_gpu(args, rank, world, local_rank):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "window": w.window, "global_batch": w.B * world, "seq_len": w.N,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between timed steps (256 MiB write, untimed)"},
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   **({"block_size": w.block_size} if w.block_size else {})},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,
@@ -395,9 +443,10 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append(v)
             samples.append(sample)
-    unit = "GB/s" if w.kind == "decode" else "TFLOP/s"
+    unit = "GB/s" if w.kind in DECODE_KINDS else "TFLOP/s"
     value = float(np.mean(vals))
-    metric = {"decode": "decode GB/s", "forward_backward": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)"} \
+    metric = {"decode": "decode GB/s", "paged_decode": "decode GB/s",
+              "forward_backward": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)"} \
         .get(w.kind, "attention TFLOP/s (fwd, unmasked FLOPs)")
     return {
         "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": 1,

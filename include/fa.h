@@ -120,6 +120,37 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode against a paged cache.  "Build a FlashAttention-2 Inference Kernel
+ * from Scratch in Pure Python", Extending It (paged KV-cache integration),
+ * read as the usual block pool: the cached rows of all sequences live in
+ * fixed-size blocks of one shared pool, and a per-sequence block table maps
+ * logical block t (keys [t * block_size, (t + 1) * block_size)) to a physical
+ * block.  Attention itself is exactly fa_decode's: query (b, h) attends to the
+ * keys j < seqlens[b] of its sequence.
+ *
+ *   q           : [B][H][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   kpool,
+ *   vpool       : [num_blocks][H][block_size][d], 16-byte aligned; key j of
+ *                 sequence b, head h is row (j mod block_size) of block
+ *                 block_table[b][j / block_size], head h.
+ *   block_table : [B][max_blocks] int32 DEVICE array.  Entries of blocks that
+ *                 hold keys j < seqlens[b] must lie in [0, num_blocks); the
+ *                 kernel checks each one it uses, skips an out-of-range block
+ *                 (never reads it) and records FA_ERR_INVALID for
+ *                 fa_get_device_status.  Other entries are never read.
+ *   seqlens     : [B] int32 DEVICE array, clamped to [0, max_blocks * block_size].
+ *   block_size  : a power of two in [1, 4096].
+ *   o, lse      : as fa_decode.
+ *   workspace   : >= fa_decode_workspace_size(B, H, max_blocks * block_size, d)
+ *                 bytes, 256-byte aligned, contents ignored on entry.
+ */
+FA_API fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool,
+                          const int32_t* block_table, const int32_t* seqlens, void* o,
+                          float* lse, int B, int H, int num_blocks, int block_size,
+                          int max_blocks, int d, float scale, fa_dtype dtype,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Decode for callers that cannot allocate device memory.  The paper has no
  * counterpart: this exists for deployment, not for the method.  Same arguments,
  * layout and results as fa_decode, minus the workspace: the per-chunk
@@ -172,8 +203,9 @@ FA_API fa_status fa_backward(const void* q, const void* k, const void* v, const 
 
 /*
  * Synchronises `stream`, then returns FA_ERR_TIMEOUT if any kernel of this
- * library recorded a barrier timeout since the last call (and clears the
- * record), FA_ERR_CUDA if the stream reports an error, else FA_OK.
+ * library recorded a barrier timeout since the last call, FA_ERR_INVALID if
+ * a paged decode met a block id outside its pool (either record is cleared),
+ * FA_ERR_CUDA if the stream reports an error, else FA_OK.
  */
 FA_API fa_status fa_get_device_status(void* stream);
 

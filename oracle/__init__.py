@@ -11,6 +11,7 @@ from .attention import (  # noqa: F401
     attention_probabilities,
     attention_scores,
     decode_forward,
+    decode_paged_forward,
     default_scale,
     merge_partials,
     online_softmax_forward,

@@ -243,6 +243,32 @@ def decode_forward(q, kcache, vcache, seqlens, scale=None):
     return o, lse
 
 
+def decode_paged_forward(q, kpool, vpool, block_table, seqlens, scale=None):
+    """Single-token decode against a paged cache.
+
+    Build a FlashAttention-2 Inference Kernel from Scratch in Pure Python,
+    Extending It (paged KV-cache integration), read as a block pool: key j of
+    sequence b, head h is row j mod bs of physical block block_table[b][j // bs]
+    of the pool.  Each sequence's keys are gathered in order and then attended
+    exactly as decode_forward does (the paging moves rows, not arithmetic).
+    kpool, vpool: [num_blocks, H, bs, d]; block_table: [B, max_blocks] ints;
+    seqlens: [B], clamped to [0, max_blocks * bs].
+    """
+    kpool, vpool = _f64(kpool), _f64(vpool)
+    table = np.asarray(block_table).astype(np.int64)
+    _, H, bs, d = kpool.shape
+    B, max_blocks = table.shape
+    cap = max_blocks * bs
+    n = np.clip(np.asarray(seqlens).astype(np.int64).reshape(-1), 0, cap)
+    kc = np.zeros((B, H, cap, d))
+    vc = np.zeros((B, H, cap, d))
+    for b in range(B):
+        for t in range(-(-int(n[b]) // bs)):
+            kc[b, :, t * bs:(t + 1) * bs] = kpool[table[b, t]]
+            vc[b, :, t * bs:(t + 1) * bs] = vpool[table[b, t]]
+    return decode_forward(q, kc, vc, n, scale)
+
+
 def merge_partials(o_parts, lse_parts):
     """Combine normalised partial results of disjoint key sets.
 

@@ -260,6 +260,35 @@ def pin_decode(o):
         assert np.abs(lse_dec[b] - lse[:, n - 1]).max() < 1e-12, b
 
 
+def pin_paged_decode(o):
+    """A padded cache cut into blocks, scattered through a pool in a random order
+    with the table recording where each block went, decodes exactly as the padded
+    cache does; table entries past a sequence's blocks (here -1) and pool rows past
+    its length (here NaN) play no part."""
+    B, H, bs, d, max_blocks = 3, 2, 4, 8, 6
+    cap = bs * max_blocks
+    seqlens = np.array([24, 9, 1])
+    kc, vc, q = _rand((B, H, cap, d), 100), _rand((B, H, cap, d), 101), _rand((B, H, d), 102)
+    o_ref, lse_ref = o.decode_forward(q, kc, vc, seqlens, 0.3)
+    nblk = [-(-int(n) // bs) for n in seqlens]
+    perm = np.random.default_rng(103).permutation(sum(nblk))
+    kpool = np.full((sum(nblk), H, bs, d), np.nan)
+    vpool = np.full((sum(nblk), H, bs, d), np.nan)
+    table = np.full((B, max_blocks), -1)
+    i = 0
+    for b in range(B):
+        for t in range(nblk[b]):
+            p = perm[i]
+            i += 1
+            table[b, t] = p
+            rows = slice(t * bs, min((t + 1) * bs, int(seqlens[b])))
+            kpool[p, :, :rows.stop - rows.start] = kc[b, :, rows]
+            vpool[p, :, :rows.stop - rows.start] = vc[b, :, rows]
+    o_pg, lse_pg = o.decode_paged_forward(q, kpool, vpool, table, seqlens, 0.3)
+    assert np.abs(o_pg - o_ref).max() < 1e-14
+    assert np.abs(lse_pg - lse_ref).max() < 1e-14
+
+
 def pin_merge(o):
     """Merging the results of disjoint key chunks (one of them empty) gives the
     result over all keys."""
@@ -303,6 +332,7 @@ ALL_PINS = [
     pin_backward_torch,
     pin_backward_identities,
     pin_decode,
+    pin_paged_decode,
     pin_merge,
     pin_rows_subset,
 ]

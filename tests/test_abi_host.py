@@ -124,3 +124,21 @@ def test_forward_backward_host_checks_its_inputs():
     q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.forward_backward_host(q, q, q, q.float())  # dout dtype differs
+
+
+def test_decode_paged_rejects_bad_arguments(lib):
+    ws = lib.fa_decode_workspace_size(2, 3, 64 * 16, 128)
+
+    def dec(table=GOOD, ws_ptr=GOOD, ws_bytes=ws, num_blocks=10, bs=16, max_blocks=64, d=128):
+        return lib.fa_decode_paged(GOOD, GOOD, GOOD, table, GOOD, GOOD, None, 2, 3, num_blocks, bs,
+                                   max_blocks, d, 0.0, fa.FA_BF16, ws_ptr, ws_bytes, None)
+
+    assert dec(table=None) == fa.FA_ERR_INVALID
+    assert dec(ws_ptr=None) == fa.FA_ERR_INVALID
+    assert dec(ws_bytes=ws - 1) == fa.FA_ERR_INVALID
+    assert dec(bs=24) == fa.FA_ERR_INVALID           # not a power of two
+    assert dec(bs=0) == fa.FA_ERR_INVALID
+    assert dec(bs=8192) == fa.FA_ERR_INVALID         # above 4096
+    assert dec(num_blocks=0) == fa.FA_ERR_INVALID
+    assert dec(max_blocks=0) == fa.FA_ERR_INVALID
+    assert dec(d=64) == fa.FA_ERR_UNSUPPORTED

@@ -50,6 +50,24 @@ def test_forward_backward_host_pipelined(chunks):
     assert_grad_close(dv, rv, f"dV chunks={chunks}")
 
 
+@pytest.mark.parametrize("causal,window", [(True, 0), (False, 90)])
+def test_autograd_binding(causal, window):
+    """fa.attention as a torch.autograd function: loss = sum(o * dO), so the
+    gradients reaching q, k, v are the backward of the forward at dO."""
+    q, k, v, dO = workloads.forward_inputs(2, 2, 200, 128, torch.bfloat16, seed=47, device="cpu",
+                                           with_dout=True)
+    qd, kd, vd = (t.cuda().requires_grad_() for t in (q, k, v))
+    o = fa.attention(qd, kd, vd, causal=causal, window=window)
+    o_ref, _ = fa.forward(qd.detach(), kd.detach(), vd.detach(), causal=causal, window=window)
+    assert torch.equal(o.detach(), o_ref)
+    (o.float() * dO.cuda().float()).sum().backward()
+    assert fa.device_status() == fa.FA_OK
+    rq, rk, rv = oracle.attention_backward(q, k, v, dO, None, causal, window)
+    assert_grad_close(qd.grad, rq, "autograd dQ")
+    assert_grad_close(kd.grad, rk, "autograd dK")
+    assert_grad_close(vd.grad, rv, "autograd dV")
+
+
 def test_backward_explicit_scale():
     q, k, v, dO = workloads.forward_inputs(2, 1, 260, 128, torch.bfloat16, seed=8, device="cpu",
                                            with_dout=True)

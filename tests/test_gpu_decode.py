@@ -77,3 +77,96 @@ def test_full_size_decode_workload_sampled():
         assert_output_close(o[b:b + 1, hs], o_ref, f"decode b={b}")
         assert_lse_close(lse[b:b + 1, hs], lse_ref, f"decode lse b={b}")
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def run_paged(q, kp, vp, table, seqlens, scale=None):
+    o, lse = fa.decode_paged(q, kp, vp, table, seqlens, scale)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("bs", [1, 16, 64, 256])
+def test_decode_paged_edge_lengths(bs):
+    """Lengths 0, 1, around a block and around the 512-key chunk, and the full
+    capacity; blocks shuffled through the pool, the unused rows of each last block
+    NaN and unused table entries -1, so any stray read shows in the output."""
+    max_blocks = -(-1100 // bs)
+    lens = [0, 1, bs - 1 if bs > 1 else 2, bs, bs + 1, 511, 512, 513, max_blocks * bs]
+    q, kp, vp, table, _ = workloads.paged_decode_inputs(len(lens), 3, bs, max_blocks, 128, 1, 1,
+                                                         seed=20 + bs, device="cpu")
+    # Re-draw a layout for these exact lengths (the generator's lengths are random).
+    g = torch.Generator().manual_seed(bs)
+    nblk = [-(-n // bs) for n in lens]
+    perm = torch.randperm(sum(nblk), generator=g)
+    kp = torch.randn(sum(nblk), 3, bs, 128, generator=g).to(torch.bfloat16)
+    vp = torch.randn(sum(nblk), 3, bs, 128, generator=g).to(torch.bfloat16)
+    table = torch.full((len(lens), max_blocks), -1, dtype=torch.int32)
+    i = 0
+    for b, n in enumerate(lens):
+        table[b, :nblk[b]] = perm[i:i + nblk[b]].to(torch.int32)
+        i += nblk[b]
+        if n % bs:
+            last = int(table[b, nblk[b] - 1])
+            kp[last, :, n % bs:] = float("nan")
+            vp[last, :, n % bs:] = float("nan")
+    seqlens = torch.tensor(lens, dtype=torch.int32)
+    o, lse = run_paged(q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), seqlens.cuda())
+    o_ref, lse_ref = oracle.decode_paged_forward(q, kp, vp, table.numpy(), seqlens.numpy(), None)
+    assert torch.all(o[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    assert_output_close(o[1:], o_ref[1:], f"paged decode O bs={bs}")
+    assert_lse_close(lse, lse_ref, f"paged decode lse bs={bs}")
+
+
+def test_decode_paged_matches_padded_cache_bitwise():
+    """The same rows as a padded cache and as a shuffled pool give identical bits:
+    only the addresses differ, the arithmetic and its order do not."""
+    B, H, bs, max_blocks = 4, 2, 32, 40
+    q, kp, vp, table, lens = workloads.paged_decode_inputs(B, H, bs, max_blocks, 128, 100, bs * max_blocks,
+                                                           seed=7, device="cuda")
+    cap = bs * max_blocks
+    kc = torch.zeros(B, H, cap, 128, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    for b in range(B):
+        for t in range(-(-int(lens[b]) // bs)):
+            kc[b, :, t * bs:(t + 1) * bs] = kp[int(table[b, t])]
+            vc[b, :, t * bs:(t + 1) * bs] = vp[int(table[b, t])]
+    o_p, lse_p = run_paged(q, kp, vp, table, lens)
+    o_c, lse_c = run_decode(q, kc, vc, lens)
+    assert torch.equal(o_p, o_c) and torch.equal(lse_p, lse_c)
+
+
+def test_decode_paged_out_of_range_block_is_reported_and_skipped():
+    """A used table entry outside the pool is never dereferenced: the kernel skips
+    that block, records FA_ERR_INVALID, and every other sequence is unaffected."""
+    B, H, bs, max_blocks = 3, 2, 16, 8
+    q, kp, vp, table, lens = workloads.paged_decode_inputs(B, H, bs, max_blocks, 128, 40, 120,
+                                                           seed=11, device="cpu")
+    bad = table.clone()
+    bad[1, 0] = kp.shape[0] + 1000
+    o, lse = fa.decode_paged(q.cuda(), kp.cuda(), vp.cuda(), bad.cuda(), lens.cuda())
+    assert fa.device_status() == fa.FA_ERR_INVALID
+    assert fa.device_status() == fa.FA_OK   # the record was cleared
+    o_ref, lse_ref = oracle.decode_paged_forward(q, kp, vp, table.numpy(), lens.numpy(), None)
+    keep = [0, 2]
+    assert_output_close(o[keep], o_ref[keep], "other sequences O")
+    assert_lse_close(lse[keep], lse_ref[keep], "other sequences lse")
+
+
+def test_full_size_paged_decode_workload_sampled():
+    """The paged decode workload at full size, in the benchmark's launch
+    configuration; the oracle checks sampled (sequence, head) pairs."""
+    w = workloads.WORKLOADS["paged_kv_decode"]
+    q, kp, vp, table, lens = workloads.workload_inputs(w, device="cuda")
+    o, lse = run_paged(q, kp, vp, table, lens, w.scale)
+    for b in (0, 17, w.B - 1):
+        nb = -(-int(lens[b]) // w.block_size)
+        tb = table[b:b + 1, :nb].cpu()
+        ids = tb[0].long()
+        sub_k, sub_v = kp[ids.cuda()].cpu(), vp[ids.cuda()].cpu()
+        local = torch.arange(nb, dtype=torch.int32).reshape(1, nb)
+        o_ref, lse_ref = oracle.decode_paged_forward(q[b:b + 1].cpu(), sub_k, sub_v, local.numpy(),
+                                                     lens[b:b + 1].cpu().numpy(), w.scale)
+        assert_output_close(o[b:b + 1], o_ref, f"paged full-size O seq {b}")
+        assert_lse_close(lse[b:b + 1], lse_ref, f"paged full-size lse seq {b}")
+    assert torch.isfinite(o.float()).all()

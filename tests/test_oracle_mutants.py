@@ -126,6 +126,23 @@ def _merge_unweighted(o_parts, lse_parts):
 
 _real_decode = om.decode_forward
 
+
+def _paged_blocks_reversed(q, kpool, vpool, block_table, seqlens, scale=None):
+    """Gathers each sequence's blocks in reverse table order."""
+    kpool, vpool = np.asarray(kpool, dtype=np.float64), np.asarray(vpool, dtype=np.float64)
+    table = np.asarray(block_table).astype(np.int64)
+    _, H, bs, d = kpool.shape
+    B, max_blocks = table.shape
+    cap = max_blocks * bs
+    n = np.clip(np.asarray(seqlens).astype(np.int64), 0, cap)
+    kc, vc = np.zeros((B, H, cap, d)), np.zeros((B, H, cap, d))
+    for b in range(B):
+        nb = -(-int(n[b]) // bs)
+        for t in range(nb):
+            kc[b, :, t * bs:(t + 1) * bs] = kpool[table[b, nb - 1 - t]]
+            vc[b, :, t * bs:(t + 1) * bs] = vpool[table[b, nb - 1 - t]]
+    return _real_decode(q, kc, vc, n, scale)
+
 MUTANTS = {
     "window_off_by_one": ("allowed_mask", _mask_window_off_by_one),
     "causal_drops_diagonal": ("allowed_mask", _mask_strict_causal),
@@ -138,6 +155,7 @@ MUTANTS = {
     "online_rescale_sign": ("online_softmax_forward", _online_sign_flip),
     "decode_reads_past_seqlen": ("decode_forward", _decode_reads_one_extra),
     "merge_unweighted": ("merge_partials", _merge_unweighted),
+    "paged_blocks_reversed": ("decode_paged_forward", _paged_blocks_reversed),
 }
 
 

@@ -44,6 +44,26 @@ def test_decode_workload_lengths_match_the_recorded_draw():
     assert int(lens.sum()) == 264373  # the seed-3 draw every decode number here is quoted on
 
 
+def test_paged_decode_inputs_place_every_block_once():
+    q, kp, vp, table, lens = workloads.paged_decode_inputs(5, 2, 16, 20, 128, 1, 300, seed=3,
+                                                           pad_value=float("nan"))
+    nblk = [(int(n) + 15) // 16 for n in lens]
+    assert kp.shape == (sum(nblk), 2, 16, 128) and table.shape == (5, 20) and table.dtype == torch.int32
+    used = torch.cat([table[b, :nblk[b]] for b in range(5)])
+    assert sorted(used.tolist()) == list(range(sum(nblk)))      # a permutation of the pool
+    for b in range(5):
+        assert (table[b, nblk[b]:] == -1).all()
+        n = int(lens[b])
+        for t in range(nblk[b]):
+            blk = kp[int(table[b, t])].float()
+            rows = min(16, n - 16 * t)
+            assert torch.isfinite(blk[:, :rows]).all() and torch.isnan(blk[:, rows:]).all()
+    # Same lengths as the padded-cache decode workload draws.
+    w = workloads.WORKLOADS["paged_kv_decode"]
+    assert torch.equal(workloads.decode_seqlens(w.B, w.seqlen_lo, w.seqlen_hi, w.seed),
+                       workloads.decode_seqlens(64, 512, 8192, 3))
+
+
 def test_named_workloads():
     W = workloads.WORKLOADS
     assert (W["single_head_fp32"].N, W["single_head_fp32"].d, W["single_head_fp32"].dtype) == (128, 64, torch.float32)
@@ -64,6 +84,12 @@ def test_flop_counts_match_closed_forms():
     assert bench.allowed_pairs(100, False, 7) == sum(100 - max(0, i - 6) for i in range(100))
     w = workloads.WORKLOADS["causal_prefill"]
     assert bench.forward_flops(w) == pytest.approx(68.753031168e9)
+    # Decode bytes: K and V rows (256 B each per head) + q + o; paged adds 4 B per used block.
+    wd, wp = workloads.WORKLOADS["kv_cache_decode"], workloads.WORKLOADS["paged_kv_decode"]
+    lens = np.array([512, 8192, 1000])
+    base = lens.sum() * 32 * 128 * 2 * 2 + 2 * 64 * 32 * 128 * 2
+    assert bench.decode_bytes(wd, lens) == base
+    assert bench.decode_bytes(wp, lens) == base + 4 * (32 + 512 + 63)
 
 
 def test_reference_arm_prints_one_json_line():

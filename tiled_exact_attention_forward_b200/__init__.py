@@ -9,10 +9,12 @@ device is missing, calls raise.
 Functions (names follow the C ABI):
     forward(q, k, v, causal=False, window=0, scale=None)        -> (o, lse)
     decode(q, kcache, vcache, seqlens, scale=None)               -> (o, lse)
+    decode_paged(q, kpool, vpool, block_table, seqlens)          -> (o, lse)
     backward(q, k, v, o, dout, lse, causal=False, window=0,
              scale=None)                                         -> (dq, dk, dv)
     forward_host(...)  -- forward on pinned host tensors (copies in and out)
     forward_backward_host(...)  -- forward and backward on pinned host tensors
+    attention(q, k, v, causal=False, window=0, scale=None)      -> o, differentiable
     device_status()    -- FA_OK or the first recorded device-side timeout
 """
 from __future__ import annotations
@@ -33,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "fa_decode_workspace_size",
     "fa_decode",
     "fa_decode_noalloc",
+    "fa_decode_paged",
     "fa_backward_workspace_size",
     "fa_backward",
     "fa_get_device_status",
@@ -72,6 +75,8 @@ def _lib() -> ctypes.CDLL:
     lib.fa_decode.restype = I
     lib.fa_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P]
     lib.fa_decode_noalloc.restype = I
+    lib.fa_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, Z, P]
+    lib.fa_decode_paged.restype = I
     lib.fa_backward_workspace_size.argtypes = [I, I, I, I]
     lib.fa_backward_workspace_size.restype = Z
     lib.fa_backward.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, I, I, P, Z, P]
@@ -281,6 +286,39 @@ def decode(q, kcache, vcache, seqlens, scale=None, workspace=None, out=None, lse
     return o, lse
 
 
+def decode_paged(q, kpool, vpool, block_table, seqlens, scale=None, workspace=None, out=None, lse=None):
+    """Single-token decode against a paged cache.
+
+    q [B, H, d]; kpool/vpool [num_blocks, H, block_size, d] (block_size a power
+    of two); block_table int32 [B, max_blocks] maps sequence b's logical block t
+    (keys [t * block_size, (t + 1) * block_size)) to a pool block; seqlens int32
+    [B].  Returns (o [B, H, d] bf16, lse [B, H] float32).  An out-of-range block
+    id of a used block is skipped and reported by device_status().
+    """
+    _need_cuda(q, kpool, vpool, block_table, seqlens)
+    B, H, d = q.shape
+    num_blocks, _, bs, _ = kpool.shape
+    if kpool.shape != (num_blocks, H, bs, d) or vpool.shape != kpool.shape:
+        raise ValueError("kpool/vpool must be [num_blocks, H, block_size, d] matching q")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be an int32 tensor of shape [B, max_blocks]")
+    if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
+        raise ValueError("seqlens must be an int32 tensor of shape [B]")
+    max_blocks = block_table.shape[1]
+    need = decode_workspace_size(B, H, max_blocks * bs, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    st = _lib().fa_decode_paged(_ptr(q), _ptr(kpool), _ptr(vpool), _ptr(block_table), _ptr(seqlens),
+                                _ptr(o), _ptr(lse), B, H, num_blocks, bs, max_blocks, d, _scale_arg(scale),
+                                _dtype_code(q.dtype), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(q.device))
+    _check(st, "fa_decode_paged")
+    return o, lse
+
+
 def backward_workspace_size(B, H, N, d) -> int:
     return int(_lib().fa_backward_workspace_size(B, H, N, d))
 
@@ -308,6 +346,34 @@ def backward(q, k, v, o, dout, lse, causal: bool = False, window: int = 0, scale
                             _stream(q.device))
     _check(st, "fa_backward")
     return dq, dk, dv
+
+
+class _Attention(torch.autograd.Function):
+    """forward keeps (q, k, v, o, lse); backward recomputes P from lse in the library."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal, window, scale):
+        o, lse = forward(q, k, v, causal, window, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.mask = (causal, window, scale)
+        return o
+
+    @staticmethod
+    def backward(ctx, grad_o):
+        q, k, v, o, lse = ctx.saved_tensors
+        causal, window, scale = ctx.mask
+        dq, dk, dv = backward(q, k, v, o, grad_o.contiguous(), lse, causal, window, scale)
+        return dq, dk, dv, None, None, None
+
+
+def attention(q, k, v, causal: bool = False, window: int = 0, scale=None):
+    """Differentiable attention: o = softmax(q k^T * scale + mask) v with autograd.
+
+    The forward runs the library's forward and saves the row logsumexp; the
+    backward runs the library's backward, which recomputes P from it (bf16,
+    d = 128 for the backward).  Gradients stay on the device.
+    """
+    return _Attention.apply(q, k, v, bool(causal), int(window), scale)
 
 
 def selftest_wait_timeout(limit_cycles: int = 20_000_000, device=None) -> int:

@@ -1,4 +1,4 @@
-// Single-token decode against a padded key/value cache (bf16, d = 128).
+// Single-token decode against a padded or a paged key/value cache (bf16, d = 128).
 //
 // "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
 // Python", Step 4: the query of (b, h) attends to every cached position
@@ -10,6 +10,11 @@
 // (o_c, lse_c).  Each half-warp owns one key row per step (16 lanes x 16
 // bytes = one 256-byte row, so a warp reads 512 contiguous bytes per load
 // instruction) and keeps 8 rows of K and 8 of V in flight per thread.
+// Paged cache ("Build a FlashAttention-2 Inference Kernel from Scratch in Pure
+// Python", Extending It: paged KV-cache integration): the rows live in
+// fixed-size blocks of a shared pool and a per-sequence block table maps the
+// logical block j / block_size to its physical block; a half-warp still reads
+// one whole 256-byte row per key, now at the table's address.
 // Combine: lse = ln sum_c exp(lse_c), o = sum_c exp(lse_c - lse) o_c -- the
 // two-softmax merge identity of "Building Flash Attention from Scratch in
 // Pure NumPy" (architecture overview), restated.
@@ -41,6 +46,7 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   }
 }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(THREADS)
     decode_split_kernel(DecodeArgs a) {
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -60,8 +66,23 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
   for (int e = 0; e < 8; ++e) qf[e] *= sl2;  // scores come out in exp2 units
 
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.kcache) + bhh * a.cap * D + sub * 8;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(a.vcache) + bhh * a.cap * D + sub * 8;
+  // Row r of the cache is at kb + r * D: r = key (contiguous) or, paged, the row of the
+  // key's physical block (the table is read per key row; rows of a block share an entry).
+  const size_t base = PAGED ? 0 : bhh * a.cap * D;
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.kcache) + base + sub * 8;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(a.vcache) + base + sub * 8;
+  const int bmask = (1 << a.block_shift) - 1;
+  bool bad_block = false;
+  // The chunk's block-table entries, staged once in shared memory so that no key
+  // row waits on a dependent table load (at most kDecodeChunk + 1 entries).
+  __shared__ int sm_blk[PAGED ? kDecodeChunk + 1 : 1];
+  const int blk0 = start >> a.block_shift;
+  if (PAGED) {
+    const int32_t* table = a.block_table + static_cast<size_t>(b) * a.max_blocks;
+    const int nblk = ((end - 1) >> a.block_shift) - blk0 + 1;
+    for (int i = threadIdx.x; i < nblk; i += THREADS) sm_blk[i] = table[blk0 + i];
+    __syncthreads();
+  }
 
   float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
@@ -73,12 +94,24 @@ __global__ void __launch_bounds__(THREADS)
   const int warp = threadIdx.x >> 5;
   for (int kbase = start + 2 * warp; kbase < end; kbase += HALVES * U) {
     uint4 kr[U], vr[U];
+    bool live[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int key = kbase + half + u * HALVES;
-      if (key < end) {
-        kr[u] = ld_stream(kb + static_cast<size_t>(key) * D);
-        vr[u] = ld_stream(vb + static_cast<size_t>(key) * D);
+      live[u] = key < end;
+      size_t r = static_cast<size_t>(key);
+      if (PAGED && live[u]) {
+        const int phys = sm_blk[(key >> a.block_shift) - blk0];
+        if (phys < 0 || phys >= a.num_blocks) {
+          bad_block = true;
+          live[u] = false;
+        } else {
+          r = ((static_cast<size_t>(phys) * a.H + h) << a.block_shift) + (key & bmask);
+        }
+      }
+      if (live[u]) {
+        kr[u] = ld_stream(kb + r * D);
+        vr[u] = ld_stream(vb + r * D);
       } else {
         kr[u] = make_uint4(0, 0, 0, 0);
         vr[u] = make_uint4(0, 0, 0, 0);
@@ -94,7 +127,7 @@ __global__ void __launch_bounds__(THREADS)
       for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      s[u] = (kbase + half + u * HALVES < end) ? dot : -INFINITY;
+      s[u] = live[u] ? dot : -INFINITY;
     }
     float mx = s[0];
 #pragma unroll
@@ -118,6 +151,8 @@ __global__ void __launch_bounds__(THREADS)
     }
     m = m_new;
   }
+
+  if (PAGED && bad_block) atomicOr(&g_status, kStatusBadBlock);
 
   // Merge the 16 half-warp states (exp2 units) through shared memory.
   __shared__ float sm_m[HALVES], sm_l[HALVES];
@@ -179,7 +214,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   using namespace dec;
   if (a.H > 65535 || a.B > 65535) return cudaErrorInvalidValue;
   dim3 grid(a.max_chunks, a.H, a.B);
-  decode_split_kernel<<<grid, THREADS, 0, stream>>>(a);
+  if (a.block_table != nullptr)
+    decode_split_kernel<true><<<grid, THREADS, 0, stream>>>(a);
+  else
+    decode_split_kernel<false><<<grid, THREADS, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<<<static_cast<unsigned>(a.B * a.H), D, 0, stream>>>(a);

@@ -100,6 +100,38 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   return from_cuda(fa::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool, const int32_t* block_table,
+                          const int32_t* seqlens, void* o, float* lse, int B, int H, int num_blocks,
+                          int block_size, int max_blocks, int d, float scale, fa_dtype dtype, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!q || !kpool || !vpool || !block_table || !seqlens || !o || !workspace) return FA_ERR_INVALID;
+  if (num_blocks < 1 || max_blocks < 1 || block_size < 1 || block_size > 4096 ||
+      (block_size & (block_size - 1)) != 0)
+    return FA_ERR_INVALID;
+  const long long cap = static_cast<long long>(max_blocks) * block_size;
+  if (!sizes_ok(B, H, cap)) return FA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(kpool, 16) || !aligned(vpool, 16) || !aligned(o, 16) ||
+      !aligned(block_table, 4) || !aligned(seqlens, 4) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID;
+  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fa_decode_workspace_size(B, H, static_cast<int>(cap), d)) return FA_ERR_INVALID;
+  fa::DecodeArgs a{};
+  a.q = q; a.kcache = kpool; a.vcache = vpool; a.seqlens = seqlens; a.o = o; a.lse = lse;
+  a.B = B; a.H = H; a.cap = static_cast<int>(cap); a.d = d;
+  a.scale = resolve_scale(scale, d);
+  a.scale_log2 = a.scale * kLog2e;
+  a.max_chunks = fa::decode_max_chunks(a.cap);
+  const size_t rows = static_cast<size_t>(B) * H * a.max_chunks;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(rows * d * sizeof(float), 256));
+  a.block_table = block_table;
+  a.block_shift = 0;
+  while ((1 << a.block_shift) < block_size) ++a.block_shift;
+  a.max_blocks = max_blocks;
+  a.num_blocks = num_blocks;
+  return from_cuda(fa::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   const size_t rows = static_cast<size_t>(B) * H * N;
@@ -148,6 +180,7 @@ fa_status fa_get_device_status(void* stream) {
     e = cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(zero));
     if (e != cudaSuccess) return FA_ERR_CUDA;
     if (word & fa::kStatusTimeout) return FA_ERR_TIMEOUT;
+    if (word & fa::kStatusBadBlock) return FA_ERR_INVALID;
   }
   return FA_OK;
 }

@@ -31,7 +31,16 @@ struct DecodeArgs {
   float* ws_o;    // [B*H][max_chunks][d] normalised chunk outputs
   float* ws_lse;  // [B*H][max_chunks] chunk logsumexp
   int max_chunks;
+  // Paged cache (block_table != null): kcache/vcache are block pools
+  // [num_blocks][H][1 << block_shift][d]; key j of sequence b sits in physical
+  // block block_table[b * max_blocks + (j >> block_shift)].  cap = max_blocks << block_shift.
+  const int32_t* block_table;
+  int block_shift, max_blocks, num_blocks;
 };
+
+// Device status bit of a paged decode that met a block id outside [0, num_blocks)
+// (the block is skipped, never read).
+constexpr unsigned kStatusBadBlock = 2u;
 
 struct BwdArgs {
   const void* q;

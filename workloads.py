@@ -9,7 +9,9 @@ Recipe: a ``torch.Generator`` seeded with the workload's seed draws, in order,
 q, k, v (and dO for the backward) as float32 standard normals, which are then
 rounded to the workload's dtype.  The decode workload first draws its
 per-sequence cache lengths from a CPU generator (uniform integers in
-[lo, hi]), then q and the two caches.  Draws on a CUDA device use torch's CUDA
+[lo, hi]), then q and the two caches; the paged decode workload draws the same
+lengths, a random placement of the blocks in the pool (CPU generator, seed + 1),
+then q and the two pools.  Draws on a CUDA device use torch's CUDA
 generator with the same seed; those values differ from the CPU stream, which
 does not matter because both sides read the same tensors.
 """
@@ -39,6 +41,7 @@ class Workload:
     window: int = 0
     seqlen_lo: int = 0   # decode only: per-sequence cache length range
     seqlen_hi: int = 0
+    block_size: int = 0  # paged decode only: rows per cache block
     notes: str = field(default="", compare=False)
 
     @property
@@ -61,6 +64,10 @@ WORKLOADS = {
                  notes="single-token decode, padded cache capacity 8192"),
         Workload("causal_fwd_bwd", "forward_backward", 2, 16, 4096, 128, BF16, 4,
                  causal=True, notes="causal forward + recompute backward"),
+        Workload("paged_kv_decode", "paged_decode", 64, 32, 8192, 128, BF16, 3,
+                 seqlen_lo=512, seqlen_hi=8192, block_size=16,
+                 notes="single-token decode against a paged cache: 16-row blocks, "
+                       "shuffled in one pool, the lengths of kv_cache_decode"),
     ]
 }
 
@@ -119,11 +126,50 @@ def decode_inputs(B, H, cap, d, lo, hi, dtype=BF16, seed=0, device="cpu",
     return q, kc, vc, seqlens.to(device)
 
 
+def paged_decode_inputs(B, H, block_size, max_blocks, d, lo, hi, dtype=BF16, seed=0, device="cpu",
+                        pad_value: float | None = None):
+    """q [B,H,d], kpool/vpool [num_blocks,H,block_size,d], block_table [B,max_blocks]
+    and seqlens [B] (int32, on ``device``).
+
+    Sequence b holds ceil(seqlens[b] / block_size) blocks; all sequences' blocks
+    are placed in one pool in a seeded random order (as a long-running cache
+    fragments), and the table maps each logical block to its place.  Table
+    entries past a sequence's blocks are -1.  Pool rows past a sequence's length
+    (the tail of its last block) are random unless ``pad_value`` is given.
+    """
+    seqlens = decode_seqlens(B, lo, hi, seed)
+    nblk = [(int(n) + block_size - 1) // block_size for n in seqlens]
+    if max(nblk) > max_blocks:
+        raise ValueError("a sequence needs more than max_blocks blocks")
+    num_blocks = max(1, sum(nblk))
+    perm = torch.randperm(num_blocks, generator=_gen(seed + 1, "cpu"))
+    table = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    first = 0
+    for b in range(B):
+        table[b, :nblk[b]] = perm[first:first + nblk[b]].to(torch.int32)
+        first += nblk[b]
+    g = _gen(seed, device)
+    q = randn((B, H, d), dtype, g, device)
+    kpool = randn((num_blocks, H, block_size, d), dtype, g, device)
+    vpool = randn((num_blocks, H, block_size, d), dtype, g, device)
+    if pad_value is not None:
+        for b in range(B):
+            n = int(seqlens[b])
+            if n % block_size:
+                last = int(table[b, nblk[b] - 1])
+                kpool[last, :, n % block_size:] = pad_value
+                vpool[last, :, n % block_size:] = pad_value
+    return q, kpool, vpool, table.to(device), seqlens.to(device)
+
+
 def workload_inputs(w: Workload, device="cpu", **kw):
     """Inputs of a named workload at its full size."""
     if w.kind == "decode":
         return decode_inputs(w.B, w.H, w.N, w.d, w.seqlen_lo, w.seqlen_hi, w.dtype,
                              w.seed, device, **kw)
+    if w.kind == "paged_decode":
+        return paged_decode_inputs(w.B, w.H, w.block_size, w.N // w.block_size, w.d, w.seqlen_lo,
+                                   w.seqlen_hi, w.dtype, w.seed, device, **kw)
     return forward_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed, device,
                           with_dout=(w.kind == "forward_backward"))
 
