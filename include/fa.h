@@ -65,7 +65,8 @@ typedef enum {
 
 typedef enum {
   FA_BF16 = 0, /* bfloat16 inputs/outputs, float32 accumulation (d = 128)   */
-  FA_FP32 = 1  /* float32 inputs/outputs, float32 arithmetic (d = 64 or 128) */
+  FA_FP32 = 1, /* float32 inputs/outputs, float32 arithmetic (d = 64 or 128) */
+  FA_FP16 = 2  /* float16 inputs/outputs, float32 accumulation (d = 128)    */
 } fa_dtype;
 
 /*
@@ -77,10 +78,11 @@ typedef enum {
  *   o       : [B][H][N][d] output (dtype), 16-byte aligned.
  *   lse     : [B][H][N] float32 output (natural-log logsumexp per row); may
  *             be NULL when the caller does not need it.
- *   B, H, N : >= 1.  d: 128 for FA_BF16; 64 or 128 for FA_FP32.
+ *   B, H, N : >= 1.  d: 128 for FA_BF16 and FA_FP16; 64 or 128 for FA_FP32.
  *   causal  : 0 or 1.  window: 0 = none, else > 0 (see Mask above).
  * Key tiles that the mask hides completely are skipped, never computed.
- * FA_BF16 runs on the tensor cores (tcgen05, TMA, TMEM); FA_FP32 on CUDA
+ * FA_BF16 and FA_FP16 run on the tensor cores (tcgen05 kind::f16 with both
+ * operands of the inputs' type, TMA, TMEM; P is formed in that type); FA_FP32 on CUDA
  * cores in float32.
  */
 FA_API fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -104,7 +106,7 @@ FA_API size_t fa_decode_workspace_size(int B, int H, int cap, int d);
  * (architecture overview): lse = ln sum_s exp(lse_s), O = sum_s
  * exp(lse_s - lse) O_s.
  *
- *   q        : [B][H][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   q        : [B][H][d] (dtype FA_BF16 or FA_FP16, d = 128), 16-byte aligned.
  *   kcache,
  *   vcache   : [B][H][cap][d], 16-byte aligned.  Rows at j >= seqlens[b]
  *              are never read.
@@ -128,7 +130,7 @@ FA_API fa_status fa_decode(const void* q, const void* kcache, const void* vcache
  * block.  Attention itself is exactly fa_decode's: query (b, h) attends to the
  * keys j < seqlens[b] of its sequence.
  *
- *   q           : [B][H][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   q           : [B][H][d] (dtype FA_BF16 or FA_FP16, d = 128), 16-byte aligned.
  *   kpool,
  *   vpool       : [num_blocks][H][block_size][d], 16-byte aligned; key j of
  *                 sequence b, head h is row (j mod block_size) of block
@@ -189,7 +191,7 @@ FA_API size_t fa_backward_workspace_size(int B, int H, int N, int d);
  * (that page's own dK/dQ lines are declared simplified; these are the exact
  * gradients of the forward).
  *
- *   q, k, v, o, dout : [B][H][N][d] (dtype FA_BF16, d = 128), 16-byte aligned.
+ *   q, k, v, o, dout : [B][H][N][d] (dtype FA_BF16 or FA_FP16, d = 128), 16-byte aligned.
  *   lse              : [B][H][N] float32 from fa_forward with the same
  *                      arguments.
  *   dq, dk, dv       : [B][H][N][d] outputs (dtype).

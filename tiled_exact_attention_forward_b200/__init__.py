@@ -28,7 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
-FA_BF16, FA_FP32 = 0, 1
+FA_BF16, FA_FP32, FA_FP16 = 0, 1, 2
 
 EXPORTED_SYMBOLS = (
     "fa_forward",
@@ -114,9 +114,11 @@ def _check(status: int, where: str):
 def _dtype_code(dt: torch.dtype) -> int:
     if dt == torch.bfloat16:
         return FA_BF16
+    if dt == torch.float16:
+        return FA_FP16
     if dt == torch.float32:
         return FA_FP32
-    raise TypeError(f"unsupported dtype {dt}: use torch.bfloat16 or torch.float32")
+    raise TypeError(f"unsupported dtype {dt}: use torch.bfloat16, torch.float16 or torch.float32")
 
 
 def _need_cuda(*ts):
@@ -134,8 +136,8 @@ def _scale_arg(scale) -> float:
 def forward(q, k, v, causal: bool = False, window: int = 0, scale=None, out=None, lse=None):
     """O = softmax(q k^T * scale + mask) v and the float32 row logsumexp.
 
-    q, k, v: [B, H, N, d] contiguous CUDA tensors (bf16 with d = 128, or fp32
-    with d in {64, 128}).  Returns (o, lse) with o like q and lse [B, H, N].
+    q, k, v: [B, H, N, d] contiguous CUDA tensors (bf16 or fp16 with d = 128, or
+    fp32 with d in {64, 128}).  Returns (o, lse) with o like q and lse [B, H, N].
     """
     _need_cuda(q, k, v)
     B, H, N, d = q.shape

@@ -1,4 +1,4 @@
-// Backward pass (bf16, d = 128) on the tensor cores.
+// Backward pass (bf16 or f16, d = 128) on the tensor cores.
 //
 // "Building Flash Attention from Scratch in Pure NumPy", Step 4: precompute
 // D = rowsum(dO * O); then for each key tile, loop over the query tiles that
@@ -9,7 +9,7 @@
 //     dS = P * (dP - D),  dK += scale * dS^T Q,  dQ += scale * dS K.
 //
 // Kernels: bwd_pre (D and zeroed fp32 dQ accumulator), bwd_main (below),
-// bwd_post (dQ fp32 -> bf16).
+// bwd_post (dQ fp32 -> the inputs' 16-bit type).
 //
 // bwd_main, one CTA per (batch*head, 128-key tile), 576 threads:
 //   * warp 17 loads K and V once, then (Q_i, dO_i) pairs by TMA into a
@@ -18,7 +18,7 @@
 //   * warps 0-7 turn S^T, dP^T into P^T and dS^T: warp w handles the key rows
 //     of TMEM lane quarter w%4 and the query columns [64h, 64h + 64),
 //     h = w/4 -- two threads per key row.  P^T and dS^T go back into tensor
-//     memory as bf16 (operands of the dV and dK MMAs) and dS^T also into
+//     memory as 16-bit pairs (operands of the dV and dK MMAs) and dS^T also into
 //     shared memory (operand of the dQ MMA);
 //   * warps 8-15 read dQ_i out of tensor memory (two threads per query row,
 //     64 columns each), stage it in shared memory (the dS buffer, free once
@@ -80,8 +80,9 @@ __device__ __forceinline__ bool tile_needs_mask(int kt, int qi, int n, int causa
 }
 
 // A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
+template <class T>
 __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t idesc = idesc_f32acc<T>(128, 128, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
@@ -90,14 +91,14 @@ __device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint
   }
 }
 
-// D[128 x d] (+)= A[tmem, 128 keys x 64 queries of half H, bf16] * B, B = [128 rows (K)][d]
+// D[128 x d] (+)= A[tmem, 128 keys x 64 queries of half H, 16-bit] * B, B = [128 rows (K)][d]
 // tile (MN-major), rows 64H .. 64H + 63.  The A columns of queries [16k, 16k + 16) sit at
-// TMEM columns 64 (k / 4) + 32 ((k % 4) / 2) + 8 (k % 2) (bf16 pairs), where the P/dS
+// TMEM columns 64 (k / 4) + 32 ((k % 4) / 2) + 8 (k % 2) (16-bit pairs), where the P/dS
 // thread that owns those queries wrote them over S^T / dP^T columns it had read.
-template <int H>
+template <int H, class T>
 __device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
                                                    bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 0, 1);
 #pragma unroll
   for (int kk = 4 * H; kk < 4 * H + 4; ++kk)
     mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8,
@@ -105,14 +106,17 @@ __device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_t
 }
 
 // dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem).
+template <class T>
 __device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+  constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < BM / 16; ++kk)
     mma_ss(d_tmem, smem_desc_sw128(ds_smem + kk * 2048, HALF_BYTES, 1024),
            smem_desc_sw128(k_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
 }
 
+// T: the 16-bit type of Q, K, V, dO, P, dS and the gradients (Bf16 or F16).
+template <class T>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -195,9 +199,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (ok) ok = mbar_wait(smem_u32(&sm.qdo_full[0]), 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_abT(tmem + T_S, ks, smem_u32(sm.q[0]));
+        issue_abT<T>(tmem + T_S, ks, smem_u32(sm.q[0]));
         tc_commit(smem_u32(&sm.s_full));
-        issue_abT(tmem + T_DP, vs, smem_u32(sm.dout[0]));
+        issue_abT<T>(tmem + T_DP, vs, smem_u32(sm.dout[0]));
         tc_commit(smem_u32(&sm.dp_full));
       }
       for (int idx = 0; ok && idx < nq; ++idx) {
@@ -208,27 +212,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = mbar_wait(smem_u32(&sm.ds_ready), 0, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_tmemA_b_half<0>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
-        issue_tmemA_b_half<0>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
+        issue_tmemA_b_half<0, T>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
+        issue_tmemA_b_half<0, T>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
         ok = mbar_wait(smem_u32(&sm.ds_ready), 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_tmemA_b_half<1>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), true);
-        issue_tmemA_b_half<1>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), true);
+        issue_tmemA_b_half<1, T>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), true);
+        issue_tmemA_b_half<1, T>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), true);
         tc_commit(smem_u32(&sm.qdo_empty[s]));
-        issue_dq(tmem + T_S, dss, ks);
+        issue_dq<T>(tmem + T_S, dss, ks);
         tc_commit(smem_u32(&sm.dq_full));
         if (idx + 1 < nq) {
           const int s1 = (idx + 1) & 1;
           ok = mbar_wait(smem_u32(&sm.qdo_full[s1]), ((idx + 1) >> 1) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_abT(tmem + T_DP, vs, smem_u32(sm.dout[s1]));
+          issue_abT<T>(tmem + T_DP, vs, smem_u32(sm.dout[s1]));
           tc_commit(smem_u32(&sm.dp_full));
           ok = mbar_wait(smem_u32(&sm.dq_free), idx & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_abT(tmem + T_S, ks, smem_u32(sm.q[s1]));
+          issue_abT<T>(tmem + T_S, ks, smem_u32(sm.q[s1]));
           tc_commit(smem_u32(&sm.s_full));
         }
       }
@@ -322,10 +326,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               pv[u] = p;
               dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
             }
-            pp[2 * e4] = pack_bf16x2(pv[0], pv[1]);
-            pp[2 * e4 + 1] = pack_bf16x2(pv[2], pv[3]);
-            dd[2 * e4] = pack_bf16x2(dsv[0], dsv[1]);
-            dd[2 * e4 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+            pp[2 * e4] = pack2<T>(pv[0], pv[1]);
+            pp[2 * e4 + 1] = pack2<T>(pv[2], pv[3]);
+            dd[2 * e4] = pack2<T>(dsv[0], dsv[1]);
+            dd[2 * e4 + 1] = pack2<T>(dsv[2], dsv[3]);
           }
           // P^T over this thread's S^T columns [8c, 8c + 8) (already read), dS^T likewise
           // over its dP^T columns.
@@ -352,7 +356,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     // Epilogue: dV rows (64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
+    uint16_t* dst = static_cast<uint16_t*>(args.dv) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
     if (ok) {
       tc_fence_after();
 #pragma unroll
@@ -369,10 +373,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint4* o4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
-            o4[v4] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v4]), __uint_as_float(r[8 * v4 + 1])),
-                                pack_bf16x2(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3])),
-                                pack_bf16x2(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])),
-                                pack_bf16x2(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7])));
+            o4[v4] = make_uint4(pack2<T>(__uint_as_float(r[8 * v4]), __uint_as_float(r[8 * v4 + 1])),
+                                pack2<T>(__uint_as_float(r[8 * v4 + 2]), __uint_as_float(r[8 * v4 + 3])),
+                                pack2<T>(__uint_as_float(r[8 * v4 + 4]), __uint_as_float(r[8 * v4 + 5])),
+                                pack2<T>(__uint_as_float(r[8 * v4 + 6]), __uint_as_float(r[8 * v4 + 7])));
         }
       }
     }
@@ -432,7 +436,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Epilogue: dK rows (scaled, 64 columns per thread).
     if (ok && nq > 0) ok = mbar_wait_warp(smem_u32(&sm.acc_done), 0, abort_flag);
     const int key = kt * BM + row;
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
+    uint16_t* dst = static_cast<uint16_t*>(args.dk) + (static_cast<size_t>(bh) * n + key) * D + 64 * hc;
     if (ok) {
       tc_fence_after();
 #pragma unroll
@@ -450,10 +454,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             o4[v4] = make_uint4(
-                pack_bf16x2(__uint_as_float(r[8 * v4]) * scale, __uint_as_float(r[8 * v4 + 1]) * scale),
-                pack_bf16x2(__uint_as_float(r[8 * v4 + 2]) * scale, __uint_as_float(r[8 * v4 + 3]) * scale),
-                pack_bf16x2(__uint_as_float(r[8 * v4 + 4]) * scale, __uint_as_float(r[8 * v4 + 5]) * scale),
-                pack_bf16x2(__uint_as_float(r[8 * v4 + 6]) * scale, __uint_as_float(r[8 * v4 + 7]) * scale));
+                pack2<T>(__uint_as_float(r[8 * v4]) * scale, __uint_as_float(r[8 * v4 + 1]) * scale),
+                pack2<T>(__uint_as_float(r[8 * v4 + 2]) * scale, __uint_as_float(r[8 * v4 + 3]) * scale),
+                pack2<T>(__uint_as_float(r[8 * v4 + 4]) * scale, __uint_as_float(r[8 * v4 + 5]) * scale),
+                pack2<T>(__uint_as_float(r[8 * v4 + 6]) * scale, __uint_as_float(r[8 * v4 + 7]) * scale));
         }
       }
     }
@@ -468,19 +472,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // D = rowsum(dO * O) in fp32 and a zeroed dQ accumulator; 16 lanes per row.
+template <class T>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, long long rows) {
   const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) >> 4;
   const int sub = threadIdx.x & 15;
   float s = 0.f;
   if (row < rows) {
-    const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.o) + row * D + sub * 8);
-    const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.dout) + row * D + sub * 8);
-    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+    float of[8], gf[8];
+    unpack8<T>(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.o) + row * D + sub * 8), of);
+    unpack8<T>(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.dout) + row * D + sub * 8), gf);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      s = fmaf(__uint_as_float(ow[i] << 16), __uint_as_float(gw[i] << 16), s);
-      s = fmaf(__uint_as_float(ow[i] & 0xffff0000u), __uint_as_float(gw[i] & 0xffff0000u), s);
-    }
+    for (int i = 0; i < 8; ++i) s = fmaf(of[i], gf[i], s);
     float4* acc = reinterpret_cast<float4*>(a.ws_dq + row * D + sub * 8);
     acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -490,41 +492,48 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(BwdArgs a, long long rows)
   if (row < rows && sub == 0) a.ws_delta[row] = s;
 }
 
-// dQ accumulator (already scaled) -> bf16; 8 elements per thread.
+// dQ accumulator (already scaled) -> T; 8 elements per thread.
+template <class T>
 __global__ void __launch_bounds__(256) bwd_post_kernel(BwdArgs a, long long n8) {
   const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
   if (i >= n8) return;
   const float4* src = reinterpret_cast<const float4*>(a.ws_dq) + 2 * i;
   const float4 x = src[0], y = src[1];
   reinterpret_cast<uint4*>(a.dq)[i] =
-      make_uint4(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w), pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+      make_uint4(pack2<T>(x.x, x.y), pack2<T>(x.z, x.w), pack2<T>(y.x, y.y), pack2<T>(y.z, y.w));
 }
 
 }  // namespace bwd
 
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+template <class T>
+cudaError_t launch_bwd_t(const BwdArgs& a, cudaStream_t stream) {
   using namespace bwd;
   const long long bh = static_cast<long long>(a.B) * a.H;
   const long long rows = bh * a.N;
   CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!make_tmap_bf16_rows(&tq, a.q, D, a.N, bh, BQ) || !make_tmap_bf16_rows(&tk, a.k, D, a.N, bh, BM) ||
-      !make_tmap_bf16_rows(&tv, a.v, D, a.N, bh, BM) || !make_tmap_bf16_rows(&tdo, a.dout, D, a.N, bh, BQ) ||
+  if (!make_tmap_half_rows(&tq, a.q, D, a.N, bh, BQ, a.f16) || !make_tmap_half_rows(&tk, a.k, D, a.N, bh, BM, a.f16) ||
+      !make_tmap_half_rows(&tv, a.v, D, a.N, bh, BM, a.f16) ||
+      !make_tmap_half_rows(&tdo, a.dout, D, a.N, bh, BQ, a.f16) ||
       !make_tmap_f32_rows(&tdq, a.ws_dq, D, a.N, bh, 32, BQ))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(bwd_main_kernel), kSmemBytes);
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(bwd_main_kernel<T>), kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long pre_blocks = (rows * 16 + 255) / 256;
   if (pre_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  bwd_pre_kernel<<<static_cast<unsigned>(pre_blocks), 256, 0, stream>>>(a, rows);
+  bwd_pre_kernel<T><<<static_cast<unsigned>(pre_blocks), 256, 0, stream>>>(a, rows);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long nkt = (a.N + BM - 1) / BM;
-  bwd_main_kernel<<<static_cast<unsigned>(nkt * bh), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
+  bwd_main_kernel<T><<<static_cast<unsigned>(nkt * bh), NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, tdo, tdq, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long n8 = rows * D / 8;
-  bwd_post_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(a, n8);
+  bwd_post_kernel<T><<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, stream>>>(a, n8);
   return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  return a.f16 ? launch_bwd_t<F16>(a, stream) : launch_bwd_t<Bf16>(a, stream);
 }
 
 }  // namespace fa

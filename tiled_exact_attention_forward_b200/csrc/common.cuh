@@ -6,6 +6,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -199,13 +200,22 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
-//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format
-//   (1 = bf16), 15 A major (0 = K), 16 B major (0 = K, 1 = MN),
+// The two 16-bit input types of kind::f16 MMAs.  One type parameter gives both
+// the A and the B format of an MMA, so a kernel never mixes them.
+struct Bf16 { static constexpr uint32_t kFormat = 1; };
+struct F16 { static constexpr uint32_t kFormat = 0; };
+
+// Instruction descriptor for kind::f16 with A and B of type T and fp32 D.
+//   bits 4-5 D format (1 = f32), 7-9 A format and 10-12 B format (0 = f16,
+//   1 = bf16), 15 A major (0 = K), 16 B major (0 = K, 1 = MN),
 //   17-22 N >> 3, 24-28 M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn_major) << 15) |
+template <class T>
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | (T::kFormat << 7) | (T::kFormat << 10) | (uint32_t(a_mn_major) << 15) |
          (uint32_t(b_mn_major) << 16) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+  return idesc_f32acc<Bf16>(M, N, a_mn_major, b_mn_major);
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
@@ -268,6 +278,38 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// The same for f16x2.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+template <class T> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<Bf16>(float lo, float hi) { return pack_bf16x2(lo, hi); }
+template <> __device__ __forceinline__ uint32_t pack2<F16>(float lo, float hi) { return pack_f16x2(lo, hi); }
+
+// Eight 16-bit values (one 16-byte load) to float.
+template <class T> __device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]);
+template <> __device__ __forceinline__ void unpack8<Bf16>(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+template <> __device__ __forceinline__ void unpack8<F16>(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] & 0xffffu)));
+    f[2 * i + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
+  }
+}
+// One float to the 16-bit type (round to nearest even), as raw bits.
+template <class T> __device__ __forceinline__ unsigned short to16(float x);
+template <> __device__ __forceinline__ unsigned short to16<Bf16>(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+template <> __device__ __forceinline__ unsigned short to16<F16>(float x) { return __half_as_ushort(__float2half_rn(x)); }
 
 // ---------------------------------------------------------------- packed fp32 (sm_100 f32x2)
 // Two floats in one 64-bit register pair; fma/add/sub/mul.rn.f32x2 process both

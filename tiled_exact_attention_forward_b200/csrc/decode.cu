@@ -1,4 +1,5 @@
-// Single-token decode against a padded or a paged key/value cache (bf16, d = 128).
+// Single-token decode against a padded or a paged key/value cache (bf16 or f16,
+// d = 128).
 //
 // "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
 // Python", Step 4: the query of (b, h) attends to every cached position
@@ -37,16 +38,8 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-
-template <bool PAGED>
+// T: the 16-bit type of q and the caches (Bf16 or F16).
+template <bool PAGED, class T>
 __global__ void __launch_bounds__(THREADS)
     decode_split_kernel(DecodeArgs a) {
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -61,7 +54,7 @@ __global__ void __launch_bounds__(THREADS)
   const size_t bhh = static_cast<size_t>(b) * a.H + h;
 
   float qf[8];
-  bf16x8_to_f32(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + bhh * D + sub * 8), qf);
+  unpack8<T>(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + bhh * D + sub * 8), qf);
   const float sl2 = a.scale_log2;
 #pragma unroll
   for (int e = 0; e < 8; ++e) qf[e] *= sl2;  // scores come out in exp2 units
@@ -69,8 +62,8 @@ __global__ void __launch_bounds__(THREADS)
   // Row r of the cache is at kb + r * D: r = key (contiguous) or, paged, the row of the
   // key's physical block (the table is read per key row; rows of a block share an entry).
   const size_t base = PAGED ? 0 : bhh * a.cap * D;
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(a.kcache) + base + sub * 8;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(a.vcache) + base + sub * 8;
+  const uint16_t* kb = static_cast<const uint16_t*>(a.kcache) + base + sub * 8;
+  const uint16_t* vb = static_cast<const uint16_t*>(a.vcache) + base + sub * 8;
   const int bmask = (1 << a.block_shift) - 1;
   bool bad_block = false;
   // The chunk's block-table entries, staged once in shared memory so that no key
@@ -121,7 +114,7 @@ __global__ void __launch_bounds__(THREADS)
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float kf[8];
-      bf16x8_to_f32(kr[u], kf);
+      unpack8<T>(kr[u], kf);
       float dot = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot = fmaf(qf[e], kf[e], dot);
@@ -145,7 +138,7 @@ __global__ void __launch_bounds__(THREADS)
       const float p = ex2_approx(s[u] - m_use);
       l += p;
       float vf[8];
-      bf16x8_to_f32(vr[u], vf);
+      unpack8<T>(vr[u], vf);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = fmaf(p, vf[e], acc[e]);
     }
@@ -182,15 +175,16 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
+template <class T>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
   const size_t bhh = blockIdx.x;
   const int b = static_cast<int>(bhh / a.H);
   const int n = min(max(a.seqlens[b], 0), a.cap);
   const int chunks = (n + kDecodeChunk - 1) / kDecodeChunk;
   const int e = threadIdx.x;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o) + bhh * D;
+  uint16_t* o = static_cast<uint16_t*>(a.o) + bhh * D;
   if (chunks == 0) {
-    o[e] = __float2bfloat16_rn(0.f);
+    o[e] = to16<T>(0.f);
     if (e == 0 && a.lse) a.lse[bhh] = -INFINITY;
     return;
   }
@@ -204,7 +198,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
     W += w;
     O = fmaf(w, os[static_cast<size_t>(c) * D + e], O);
   }
-  o[e] = __float2bfloat16_rn(O / W);
+  o[e] = to16<T>(O / W);
   if (e == 0 && a.lse) a.lse[bhh] = M + logf(W);
 }
 
@@ -215,12 +209,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (a.H > 65535 || a.B > 65535) return cudaErrorInvalidValue;
   dim3 grid(a.max_chunks, a.H, a.B);
   if (a.block_table != nullptr)
-    decode_split_kernel<true><<<grid, THREADS, 0, stream>>>(a);
+    (a.f16 ? decode_split_kernel<true, F16> : decode_split_kernel<true, Bf16>)<<<grid, THREADS, 0, stream>>>(a);
   else
-    decode_split_kernel<false><<<grid, THREADS, 0, stream>>>(a);
+    (a.f16 ? decode_split_kernel<false, F16> : decode_split_kernel<false, Bf16>)<<<grid, THREADS, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<static_cast<unsigned>(a.B * a.H), D, 0, stream>>>(a);
+  (a.f16 ? decode_combine_kernel<F16> : decode_combine_kernel<Bf16>)<<<static_cast<unsigned>(a.B * a.H), D, 0, stream>>>(a);
   return cudaGetLastError();
 }
 

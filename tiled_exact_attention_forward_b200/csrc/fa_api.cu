@@ -59,8 +59,9 @@ fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float
   a.scale = resolve_scale(scale, d);
   a.scale_log2 = a.scale * kLog2e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16) {
+  if (dtype == FA_BF16 || dtype == FA_FP16) {
     if (d != 128) return FA_ERR_UNSUPPORTED;
+    a.f16 = dtype == FA_FP16;
     return from_cuda(fa::launch_fwd_tc(a, st));
   }
   if (dtype == FA_FP32) {
@@ -85,7 +86,7 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
       !aligned(seqlens, 4) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
     return FA_ERR_INVALID;
-  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if ((dtype != FA_BF16 && dtype != FA_FP16) || d != 128) return FA_ERR_UNSUPPORTED;
   if (workspace_bytes < fa_decode_workspace_size(B, H, cap, d)) return FA_ERR_INVALID;
   fa::DecodeArgs a{};
   a.q = q; a.kcache = kcache; a.vcache = vcache; a.seqlens = seqlens; a.o = o; a.lse = lse;
@@ -93,6 +94,7 @@ fa_status fa_decode(const void* q, const void* kcache, const void* vcache, const
   a.scale = resolve_scale(scale, d);
   a.scale_log2 = a.scale * kLog2e;
   a.max_chunks = fa::decode_max_chunks(cap);
+  a.f16 = dtype == FA_FP16;
   const size_t rows = static_cast<size_t>(B) * H * a.max_chunks;
   a.ws_o = static_cast<float*>(workspace);
   a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -113,7 +115,7 @@ fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool, c
   if (!aligned(q, 16) || !aligned(kpool, 16) || !aligned(vpool, 16) || !aligned(o, 16) ||
       !aligned(block_table, 4) || !aligned(seqlens, 4) || !aligned(workspace, 256) || (lse && !aligned(lse, 4)))
     return FA_ERR_INVALID;
-  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if ((dtype != FA_BF16 && dtype != FA_FP16) || d != 128) return FA_ERR_UNSUPPORTED;
   if (workspace_bytes < fa_decode_workspace_size(B, H, static_cast<int>(cap), d)) return FA_ERR_INVALID;
   fa::DecodeArgs a{};
   a.q = q; a.kcache = kpool; a.vcache = vpool; a.seqlens = seqlens; a.o = o; a.lse = lse;
@@ -121,6 +123,7 @@ fa_status fa_decode_paged(const void* q, const void* kpool, const void* vpool, c
   a.scale = resolve_scale(scale, d);
   a.scale_log2 = a.scale * kLog2e;
   a.max_chunks = fa::decode_max_chunks(a.cap);
+  a.f16 = dtype == FA_FP16;
   const size_t rows = static_cast<size_t>(B) * H * a.max_chunks;
   a.ws_o = static_cast<float*>(workspace);
   a.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(rows * d * sizeof(float), 256));
@@ -148,7 +151,7 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   for (const void* p : ptrs16)
     if (!aligned(p, 16)) return FA_ERR_INVALID;
   if (!aligned(lse, 4) || !aligned(workspace, 256)) return FA_ERR_INVALID;
-  if (dtype != FA_BF16 || d != 128) return FA_ERR_UNSUPPORTED;
+  if ((dtype != FA_BF16 && dtype != FA_FP16) || d != 128) return FA_ERR_UNSUPPORTED;
   if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID;
   fa::BwdArgs a{};
   a.q = q; a.k = k; a.v = v; a.o = o; a.dout = dout; a.lse = lse;
@@ -157,6 +160,7 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   a.causal = causal; a.window = window;
   a.scale = resolve_scale(scale, d);
   a.scale_log2 = a.scale * kLog2e;
+  a.f16 = dtype == FA_FP16;
   const size_t rows = static_cast<size_t>(B) * H * N;
   a.ws_delta = static_cast<float*>(workspace);
   a.ws_dq = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(rows * sizeof(float), 256));

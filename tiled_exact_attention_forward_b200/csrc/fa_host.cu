@@ -29,8 +29,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_head, long long heads,
-                         int box_rows) {
+bool make_tmap_half_rows(void* map, const void* base, int d, long long rows_per_head, long long heads,
+                         int box_rows, int f16) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows_per_head),
@@ -39,7 +39,8 @@ bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_
                            static_cast<cuuint64_t>(d) * 2 * static_cast<cuuint64_t>(rows_per_head)};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  CUresult r = fn(reinterpret_cast<CUtensorMap*>(map),
+                  f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                   const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

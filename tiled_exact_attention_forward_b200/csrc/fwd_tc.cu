@@ -1,4 +1,5 @@
-// Forward pass on the 5th-generation tensor cores (sm_100a): tcgen05 MMAs with
+// Forward pass on the 5th-generation tensor cores (sm_100a), bf16 or f16 inputs
+// (one kernel template; P is formed in the inputs' type): tcgen05 MMAs with
 // fp32 accumulators in tensor memory, K/V tiles streamed by TMA through a
 // shared-memory ring, and the online softmax in registers.
 //
@@ -31,7 +32,7 @@
 //     measured slower: the two softmaxes then overlap and contend for the
 //     same pipes, where the fixed order below keeps them alternating.)
 //   * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
-//     The softmax writes P (bf16 pairs) over the first 64 columns of its S
+//     The softmax writes P (16-bit pairs) over the first 64 columns of its S
 //     tile, and O += P V reads P straight from tensor memory (A operand in
 //     TMEM), so P never touches shared memory.
 //   * MMA issue order per key tile j (ping-pong):
@@ -58,7 +59,7 @@ constexpr int BM = 128;                 // query rows per tile
 constexpr int BN = 128;                 // keys per tile
 constexpr int D = 128;                  // head dimension
 constexpr int NS = 4;                   // K/V ring stages (K and V tiles interleaved)
-constexpr int TILE_BYTES = BM * D * 2;  // one 128 x 128 bf16 tile = 32 KiB
+constexpr int TILE_BYTES = BM * D * 2;  // one 128 x 128 16-bit tile = 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;  // one 64-column half (a 128-byte-swizzled box)
 constexpr int NUM_THREADS = 608;     // 16 softmax warps + MMA warp + K/V TMA warp + Q TMA warp
 constexpr int WG_THREADS = 256;      // one softmax warpgroup pair per query tile
@@ -121,8 +122,9 @@ __device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
 
 // S = Q K^T: Q and K tiles K-major ([64-column half][128 rows][64 cols]); a K step
 // of 16 columns is 32 bytes inside a half, the second half 16 KiB further on.
+template <class T>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
-  constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+  constexpr uint32_t idesc = idesc_f32acc<T>(BM, BN, 0, 0);
   constexpr uint32_t hi = desc_hi(1024);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
@@ -133,9 +135,10 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_
 
 // O += P V: V tile MN-major ([64-column half][128 keys][64 cols]); a K step of 16
 // keys is 16 rows = 2 KiB.  P of keys [64h, 64h + 64) sits in S columns
-// [64h, 64h + 32) (bf16 pairs).
+// [64h, 64h + 32) (16-bit pairs).
+template <class T>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo, bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+  constexpr uint32_t idesc = idesc_f32acc<T>(BM, D, 0, 1);
   constexpr uint32_t hi = desc_hi(1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
@@ -185,6 +188,8 @@ __device__ __forceinline__ int item_of(int k, int total) {
   return lin < total ? lin : -1;
 }
 
+// T: the 16-bit type of Q, K, V, P and O (Bf16 or F16).
+template <class T>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, FwdArgs args) {
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           q_ready[t] = true;
           tc_fence_after();
         }
-        issue_qk(tS[t], q_s[t], ks);
+        issue_qk<T>(tS[t], q_s[t], ks);
         tc_commit(smem_u32(&sm.s_full[t]));
         if (j == it.hi_t[t] - 1) {
           tc_commit(smem_u32(&sm.q_empty[t]));
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (!mbar_wait(smem_u32(&sm.p_full[t]), npv[t] & 1, abort_flag)) return false;
           tc_fence_after();
-          issue_pv(tO[t], tS[t], vs, j > it.lo_t[t]);
+          issue_pv<T>(tO[t], tS[t], vs, j > it.lo_t[t]);
           ++npv[t];
           if (j == it.hi_t[t] - 1) {
             tc_commit(smem_u32(&sm.o_full[t]));
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           l *= alpha;
         }
         const float ms = (m == -INFINITY) ? 0.f : m * sl2;
-        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> bf16 pairs over this
+        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> 16-bit pairs over this
         // half's first 32 S columns (already read).  Scores go in pairs through the
         // packed f32x2 FMA; kPolyPairs of every 8 pairs take 2^x from the cubic on
         // the FMA pipe, the rest from the special-function unit, so both pipes share
@@ -498,7 +503,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (e & 2) acc_b = f2_add(acc_b, p2); else acc_a = f2_add(acc_a, p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
-            p[e >> 1] = pack_bf16x2(p0, p1);
+            p[e >> 1] = pack2<T>(p0, p1);
           }
           asm volatile(
               "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -530,7 +535,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!ok) break;
-      // Epilogue: O / l in bf16 and lse = m * scale + ln l.  O_t is read out first and
+      // Epilogue: O / l in 16 bits and lse = m * scale + ln l.  O_t is read out first and
       // released (o_free) so the next item's PV can start while the stores drain.
       ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nout & 1, abort_flag);
       ++nout;
@@ -549,16 +554,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (nan_row) lt = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
       const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
       if (row_g < n) {
-        __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
+        uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) +
                               (static_cast<size_t>(item.bh) * n + row_g) * D + 64 * hc;
         uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
         for (int v4 = 0; v4 < 8; ++v4) {
           uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+          w.x = pack2<T>(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+          w.y = pack2<T>(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+          w.z = pack2<T>(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+          w.w = pack2<T>(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
           dst[v4] = w;
         }
         if (hc == 0 && args.lse != nullptr)
@@ -581,19 +586,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   using namespace fwdtc;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_bf16_rows(&tq, a.q, D, a.N, static_cast<long long>(a.B) * a.H, BM) ||
-      !make_tmap_bf16_rows(&tk, a.k, D, a.N, static_cast<long long>(a.B) * a.H, BN) ||
-      !make_tmap_bf16_rows(&tv, a.v, D, a.N, static_cast<long long>(a.B) * a.H, BN))
+  const long long heads = static_cast<long long>(a.B) * a.H;
+  if (!make_tmap_half_rows(&tq, a.q, D, a.N, heads, BM, a.f16) ||
+      !make_tmap_half_rows(&tk, a.k, D, a.N, heads, BN, a.f16) ||
+      !make_tmap_half_rows(&tv, a.v, D, a.N, heads, BN, a.f16))
     return cudaErrorInvalidValue;
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(fwd_tc_kernel), kSmemBytes);
+  auto kernel = a.f16 ? fwd_tc_kernel<F16> : fwd_tc_kernel<Bf16>;
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
-  const long long items = static_cast<long long>((a.N + 2 * BM - 1) / (2 * BM)) * a.B * a.H;
+  const long long items = static_cast<long long>((a.N + 2 * BM - 1) / (2 * BM)) * heads;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
   int sms = 0;
   e = sm_count(&sms);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  fwd_tc_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, a);
+  kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
 

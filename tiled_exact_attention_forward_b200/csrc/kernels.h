@@ -17,6 +17,7 @@ struct FwdArgs {
   int causal, window;
   float scale;       // natural units
   float scale_log2;  // scale * log2(e)
+  int f16;           // 16-bit inputs/outputs are f16 (else bf16)
 };
 
 struct DecodeArgs {
@@ -36,6 +37,7 @@ struct DecodeArgs {
   // block block_table[b * max_blocks + (j >> block_shift)].  cap = max_blocks << block_shift.
   const int32_t* block_table;
   int block_shift, max_blocks, num_blocks;
+  int f16;  // q, caches and o are f16 (else bf16)
 };
 
 // Device status bit of a paged decode that met a block id outside [0, num_blocks)
@@ -57,6 +59,7 @@ struct BwdArgs {
   float scale, scale_log2;
   float* ws_delta;  // [B*H*N] rowsum(dO * O)
   float* ws_dq;     // [B*H*N*d] fp32 dQ accumulator
+  int f16;          // 16-bit tensors are f16 (else bf16)
 };
 
 // Decode: keys per split chunk (one CTA each).
@@ -65,10 +68,11 @@ constexpr int kDecodeChunk = 512;
 inline int decode_max_chunks(int cap) { return (cap + kDecodeChunk - 1) / kDecodeChunk; }
 
 // Host helpers (fa_host.cu).
-// A 3-D TMA map over a bf16 [heads][rows_per_head][d] array: boxes of 64
-// columns x box_rows rows, 128-byte swizzle, rows past the end read as zero.
-bool make_tmap_bf16_rows(void* map, const void* base, int d, long long rows_per_head,
-                         long long heads, int box_rows);
+// A 3-D TMA map over a 16-bit (bf16, or f16 when f16 != 0) [heads][rows_per_head][d]
+// array: boxes of 64 columns x box_rows rows, 128-byte swizzle, rows past the end
+// read as zero.
+bool make_tmap_half_rows(void* map, const void* base, int d, long long rows_per_head,
+                         long long heads, int box_rows, int f16);
 // The same over a float32 array, boxes of box_cols (32: 128 bytes) x box_rows.
 bool make_tmap_f32_rows(void* map, const void* base, int d, long long rows_per_head,
                         long long heads, int box_cols, int box_rows);

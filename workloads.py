@@ -64,6 +64,8 @@ WORKLOADS = {
                  notes="single-token decode, padded cache capacity 8192"),
         Workload("causal_fwd_bwd", "forward_backward", 2, 16, 4096, 128, BF16, 4,
                  causal=True, notes="causal forward + recompute backward"),
+        Workload("causal_prefill_fp16", "forward", 4, 16, 2048, 128, torch.float16, 1, causal=True,
+                 notes="the causal prefill forward with float16 inputs"),
         Workload("paged_kv_decode", "paged_decode", 64, 32, 8192, 128, BF16, 3,
                  seqlen_lo=512, seqlen_hi=8192, block_size=16,
                  notes="single-token decode against a paged cache: 16-row blocks, "
