@@ -118,9 +118,10 @@ def test_decode_paged_edge_lengths(bs):
     assert_lse_close(lse, lse_ref, f"paged decode lse bs={bs}")
 
 
-def test_decode_paged_matches_padded_cache_bitwise():
-    """The same rows as a padded cache and as a shuffled pool give identical bits:
-    only the addresses differ, the arithmetic and its order do not."""
+def test_decode_paged_matches_padded_cache():
+    """The same rows as a padded cache and as a shuffled pool give the same result up
+    to the order of the final merge (paged decode splits the keys into 1024-key
+    chunks, padded decode into 512-key chunks)."""
     B, H, bs, max_blocks = 4, 2, 32, 40
     q, kp, vp, table, lens = workloads.paged_decode_inputs(B, H, bs, max_blocks, 128, 100, bs * max_blocks,
                                                            seed=7, device="cuda")
@@ -133,7 +134,8 @@ def test_decode_paged_matches_padded_cache_bitwise():
             vc[b, :, t * bs:(t + 1) * bs] = vp[int(table[b, t])]
     o_p, lse_p = run_paged(q, kp, vp, table, lens)
     o_c, lse_c = run_decode(q, kc, vc, lens)
-    assert torch.equal(o_p, o_c) and torch.equal(lse_p, lse_c)
+    assert (o_p.float() - o_c.float()).abs().max() <= 2 ** -8
+    assert (lse_p - lse_c).abs().max() <= 1e-5
 
 
 def test_decode_paged_out_of_range_block_is_reported_and_skipped():

@@ -6,8 +6,8 @@
 // j < seqlens[b] (the cache already holds the current token).  The work is
 // HBM-bound: every cached key and value row is read once, 256 bytes each.
 //
-// Split: CTA (chunk, h, b) scores keys [chunk * 512, chunk * 512 + 512) of
-// its sequence with the online softmax and writes a normalised partial
+// Split: CTA (chunk, h, b) scores keys [chunk * 512, chunk * 512 + 512) (paged:
+// 1024-key chunks) of its sequence with the online softmax and writes a normalised partial
 // (o_c, lse_c).  Each half-warp owns one key row per step (16 lanes x 16
 // bytes = one 256-byte row, so a warp reads 512 contiguous bytes per load
 // instruction) and keeps 8 rows of K and 8 of V in flight per thread.
@@ -29,6 +29,9 @@ constexpr int D = 128;
 constexpr int THREADS = 256;          // 8 warps = 16 half-warps
 constexpr int HALVES = THREADS / 16;
 constexpr int U = 8;                  // key rows in flight per half-warp and step
+// Keys per split CTA: a paged CTA first loads its chunk's block-table entries, a
+// dependent load before its first row, so it takes twice the keys to amortise it.
+template <bool PAGED> __host__ __device__ constexpr int chunk_keys() { return PAGED ? 2 * kDecodeChunk : kDecodeChunk; }
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
@@ -44,9 +47,10 @@ __global__ void __launch_bounds__(THREADS)
     decode_split_kernel(DecodeArgs a) {
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int n = min(max(a.seqlens[b], 0), a.cap);
-  const int start = c * kDecodeChunk;
+  constexpr int CHUNK = chunk_keys<PAGED>();
+  const int start = c * CHUNK;
   if (start >= n) return;
-  const int end = min(start + kDecodeChunk, n);
+  const int end = min(start + CHUNK, n);
 
   const int lane = threadIdx.x & 31;
   const int hw = threadIdx.x >> 4;   // half-warp 0..15 (keys start + hw + 16 i)
@@ -67,8 +71,8 @@ __global__ void __launch_bounds__(THREADS)
   const int bmask = (1 << a.block_shift) - 1;
   bool bad_block = false;
   // The chunk's block-table entries, staged once in shared memory so that no key
-  // row waits on a dependent table load (at most kDecodeChunk + 1 entries).
-  __shared__ int sm_blk[PAGED ? kDecodeChunk + 1 : 1];
+  // row waits on a dependent table load (at most CHUNK + 1 entries).
+  __shared__ int sm_blk[PAGED ? CHUNK + 1 : 1];
   const int blk0 = start >> a.block_shift;
   if (PAGED) {
     const int32_t* table = a.block_table + static_cast<size_t>(b) * a.max_blocks;
@@ -175,12 +179,13 @@ __global__ void __launch_bounds__(THREADS)
   }
 }
 
-template <class T>
+template <bool PAGED, class T>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
   const size_t bhh = blockIdx.x;
   const int b = static_cast<int>(bhh / a.H);
   const int n = min(max(a.seqlens[b], 0), a.cap);
-  const int chunks = (n + kDecodeChunk - 1) / kDecodeChunk;
+  constexpr int CHUNK = chunk_keys<PAGED>();
+  const int chunks = (n + CHUNK - 1) / CHUNK;
   const int e = threadIdx.x;
   uint16_t* o = static_cast<uint16_t*>(a.o) + bhh * D;
   if (chunks == 0) {
@@ -207,14 +212,21 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   using namespace dec;
   if (a.H > 65535 || a.B > 65535) return cudaErrorInvalidValue;
-  dim3 grid(a.max_chunks, a.H, a.B);
-  if (a.block_table != nullptr)
+  // a.max_chunks counts kDecodeChunk-key chunks (it sizes the workspace); a paged
+  // CTA takes two of them.
+  const bool paged = a.block_table != nullptr;
+  const dim3 grid(paged ? (a.max_chunks + 1) / 2 : a.max_chunks, a.H, a.B);
+  if (paged)
     (a.f16 ? decode_split_kernel<true, F16> : decode_split_kernel<true, Bf16>)<<<grid, THREADS, 0, stream>>>(a);
   else
     (a.f16 ? decode_split_kernel<false, F16> : decode_split_kernel<false, Bf16>)<<<grid, THREADS, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  (a.f16 ? decode_combine_kernel<F16> : decode_combine_kernel<Bf16>)<<<static_cast<unsigned>(a.B * a.H), D, 0, stream>>>(a);
+  const unsigned rows = static_cast<unsigned>(a.B * a.H);
+  if (paged)
+    (a.f16 ? decode_combine_kernel<true, F16> : decode_combine_kernel<true, Bf16>)<<<rows, D, 0, stream>>>(a);
+  else
+    (a.f16 ? decode_combine_kernel<false, F16> : decode_combine_kernel<false, Bf16>)<<<rows, D, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
