@@ -92,12 +92,13 @@ def test_flop_counts_match_closed_forms():
     assert bench.decode_bytes(wp, lens) == base + 4 * (32 + 512 + 63)
 
 
-def test_reference_arm_prints_one_json_line():
+@pytest.mark.parametrize("workload,unit", [("single_head_fp32", "TFLOP/s"), ("paged_kv_decode", "GB/s")])
+def test_reference_arm_prints_one_json_line(workload, unit):
     env = dict(os.environ)
     env.pop("RANK", None)
     env.pop("WORLD_SIZE", None)
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                        "--warmup", "3", "--ref-budget", "0.5", "--workload", "single_head_fp32"],
+                        "--warmup", "3", "--ref-budget", "0.5", "--workload", workload],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
@@ -106,6 +107,7 @@ def test_reference_arm_prints_one_json_line():
     for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "cpu_baseline",
                 "e2e", "config"):
         assert key in d, key
-    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == unit
+    assert d["config"]["workload"] == workload
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert np.isfinite(d["value"])
