@@ -12,14 +12,17 @@
  *     Step 3 (the forward's tile loops and its scale=None default), Step 4
  *     (the backward from the saved row statistics, D = rowsum(dO * O)).
  *   - "Build a FlashAttention-2 Inference Kernel from Scratch in Pure Python":
- *     Steps 2-3 (scale, mask to -inf, causal j <= i, sliding-window skipping).
+ *     Steps 2-3 (scale, mask to -inf, causal j <= i, sliding-window skipping);
+ *     Extending It (paged KV-cache integration, read as a block pool).
  *   - "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
  *     Python": Step 4 (single-query decode against a key/value cache).
  *
  * Conventions shared by every entry point
  *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major
  *     [B][H][N][d] (d innermost).  lse is float32 [B][H][N].  Decode: q and o
- *     are [B][H][d], the caches [B][H][cap][d], seqlens int32 [B].
+ *     are [B][H][d], the caches [B][H][cap][d], seqlens int32 [B]; paged
+ *     decode: pools [num_blocks][H][block_size][d], block table int32
+ *     [B][max_blocks].
  *   - Mask: key j is visible to query i iff
  *         (causal == 0 || j <= i) && (window <= 0 || j > i - window),
  *     so a window holds exactly `window` keys including the query itself.
@@ -36,8 +39,9 @@
  *     workspace too small, window < 0) or FA_ERR_UNSUPPORTED (a dtype/d
  *     combination with no kernel).  FA_ERR_CUDA reports a failed launch.
  *   - Kernels never trap.  A kernel that waits too long on an internal
- *     barrier records FA_ERR_TIMEOUT in a device status word and returns;
- *     fa_get_device_status() reports it.
+ *     barrier records FA_ERR_TIMEOUT in a device status word and returns; a
+ *     paged decode that meets a block id outside its pool skips that block and
+ *     records FA_ERR_INVALID; fa_get_device_status() reports either.
  */
 #ifndef TILED_EXACT_ATTENTION_FA_H_
 #define TILED_EXACT_ATTENTION_FA_H_

@@ -37,7 +37,7 @@ def test_status_strings_and_version(lib):
     for code in range(5):
         assert lib.fa_status_string(code).startswith(b"FA_")
     assert lib.fa_status_string(99) == b"unknown fa_status"
-    assert lib.fa_version() == 100
+    assert lib.fa_version() == 101  # 1.01: fa_decode_paged and FA_FP16 added to 1.00
 
 
 P = ctypes.c_void_p

@@ -32,7 +32,7 @@ bool sizes_ok(long long B, long long H, long long N) {
 
 extern "C" {
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 101; }
 
 const char* fa_status_string(fa_status s) {
   switch (s) {
