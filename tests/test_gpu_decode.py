@@ -172,3 +172,15 @@ def test_full_size_paged_decode_workload_sampled():
         assert_output_close(o[b:b + 1], o_ref, f"paged full-size O seq {b}")
         assert_lse_close(lse[b:b + 1], lse_ref, f"paged full-size lse seq {b}")
     assert torch.isfinite(o.float()).all()
+
+
+def test_decode_bindings_reject_mismatched_dtypes():
+    """A cache of another dtype than q is refused before any launch."""
+    q = torch.zeros(1, 2, 128, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(1, 2, 64, 128, dtype=torch.float16, device="cuda")
+    lens = torch.full((1,), 64, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        fa.decode(q, kc, kc, lens)
+    table = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        fa.decode_paged(q, kc.view(4, 2, 16, 128), kc.view(4, 2, 16, 128), table, lens)

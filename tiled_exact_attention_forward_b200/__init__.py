@@ -127,6 +127,8 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
+        if t.device != ts[0].device:
+            raise ValueError("tensors must all be on the same CUDA device")
 
 
 def _scale_arg(scale) -> float:
@@ -272,6 +274,8 @@ def decode(q, kcache, vcache, seqlens, scale=None, workspace=None, out=None, lse
     cap = kcache.shape[2]
     if kcache.shape != (B, H, cap, d) or vcache.shape != kcache.shape:
         raise ValueError("kcache/vcache must be [B, H, cap, d] matching q")
+    if kcache.dtype != q.dtype or vcache.dtype != q.dtype:
+        raise ValueError("kcache/vcache must have q's dtype")
     if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
         raise ValueError("seqlens must be an int32 tensor of shape [B]")
     need = decode_workspace_size(B, H, cap, d)
@@ -302,6 +306,8 @@ def decode_paged(q, kpool, vpool, block_table, seqlens, scale=None, workspace=No
     num_blocks, _, bs, _ = kpool.shape
     if kpool.shape != (num_blocks, H, bs, d) or vpool.shape != kpool.shape:
         raise ValueError("kpool/vpool must be [num_blocks, H, block_size, d] matching q")
+    if kpool.dtype != q.dtype or vpool.dtype != q.dtype:
+        raise ValueError("kpool/vpool must have q's dtype")
     if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError("block_table must be an int32 tensor of shape [B, max_blocks]")
     if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
