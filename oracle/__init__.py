@@ -7,6 +7,7 @@ from .attention import (  # noqa: F401
     allowed_mask,
     attention_backward,
     attention_forward,
+    attention_forward_offset,
     attention_forward_rows,
     attention_probabilities,
     attention_scores,

@@ -19,6 +19,10 @@ eye.  Sources (web pages, cited by title and section):
 * "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
   Python" -- Steps 2-5 (single-query decode against a cache that already holds
   the current token; naive single-query reference).
+* The same two pages' "Extending It" roadmaps (distributed tensor
+  parallelism; horizontal scaling with each worker holding part of the
+  key/value space): the per-shard partial forward of
+  :func:`attention_forward_offset`, combined with :func:`merge_partials`.
 * "FlashAttention Algorithm > Worked Example" -- the n=8, d=4, block 4 trace
   (Steps 1-3) that pins :func:`online_softmax_forward` and
   :func:`attention_forward`.
@@ -65,6 +69,7 @@ __all__ = [
     "attention_probabilities",
     "attention_forward",
     "attention_forward_rows",
+    "attention_forward_offset",
     "attention_backward",
     "decode_forward",
     "merge_partials",
@@ -267,6 +272,27 @@ def decode_paged_forward(q, kpool, vpool, block_table, seqlens, scale=None):
             kc[b, :, t * bs:(t + 1) * bs] = kpool[table[b, t]]
             vc[b, :, t * bs:(t + 1) * bs] = vpool[table[b, t]]
     return decode_forward(q, kc, vc, n, scale)
+
+
+def attention_forward_offset(q, k, v, q_offset, scale=None, causal=False, window=0):
+    """One key shard's partial forward, for context-parallel attention, in float64.
+
+    Build a FlashAttention-2 Inference Kernel from Scratch in Pure Python,
+    "Extending It" (distributed tensor parallelism: the attention matrix split
+    across devices so the context outgrows one device's memory), and Build a
+    FlashAttention Kernel with Online Softmax and KV Cache in Pure Python,
+    "Extending It" (horizontal scaling: each worker holds a portion of the
+    key/value space).  Reading: a worker holding a contiguous run of keys
+    computes the softmax over its own keys only, with the causal and window
+    masks evaluated at sequence positions -- query row i sits ``q_offset + i``
+    positions after the shard's first key.  Rows that see no key of the shard
+    get O = 0 and lse = -inf; the partials of all shards combine into the full
+    result with :func:`merge_partials`.
+    q: [..., Nq, d]; k, v: [..., Nk, d].  Returns (O [..., Nq, d], lse [..., Nq]).
+    """
+    q_pos = int(q_offset) + np.arange(np.asarray(q.shape)[-2])
+    P, lse = attention_probabilities(q, k, scale, causal, window, q_pos=q_pos)
+    return np.matmul(P, _f64(v)), lse
 
 
 def merge_partials(o_parts, lse_parts):

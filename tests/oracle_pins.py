@@ -320,6 +320,62 @@ def pin_rows_subset(o):
         assert np.abs(lr - lse[rows]).max() < 1e-14
 
 
+def pin_offset_shards(o):
+    """Context parallelism: cut a ragged sequence into query and key shards of
+    unequal length; each query shard's partials against every key shard, with
+    the offset between the shards' first positions, merge into the same rows of
+    the full forward.  Shards that a query shard cannot see come back empty
+    (lse = -inf) and drop out of the merge."""
+    N, d = 37, 4
+    q, k, v = _rand((2, N, d), 120), _rand((2, N, d), 121), _rand((2, N, d), 122)
+    bounds = [(0, 10), (10, 11), (11, 23), (23, 37)]
+    for causal, window in MASKS + [(True, 12), (False, 30)]:
+        O, lse = o.attention_forward(q, k, v, 0.4, causal, window)
+        for qlo, qhi in bounds:
+            parts_o, parts_l = [], []
+            for klo, khi in bounds:
+                po, pl = o.attention_forward_offset(q[:, qlo:qhi], k[:, klo:khi], v[:, klo:khi],
+                                                    qlo - klo, 0.4, causal, window)
+                parts_o.append(po)
+                parts_l.append(pl)
+            Om, lm = o.merge_partials(np.stack(parts_o), np.stack(parts_l))
+            assert np.abs(Om - O[:, qlo:qhi]).max() < 1e-12, (causal, window, qlo)
+            assert np.abs(lm - lse[:, qlo:qhi]).max() < 1e-12, (causal, window, qlo)
+
+
+def pin_offset_closed_form(o):
+    """q = 0 makes every visible score 0: with query row i at position off + i,
+    O_i is the mean of the V rows it sees and lse_i = ln(their count); a row
+    that sees none gets O = 0 and lse = -inf.  Also checked against torch's
+    float64 scaled_dot_product_attention on random inputs, with the mask built
+    from positions by loops."""
+    Nq, Nk, d = 6, 9, 3
+    k, v = _rand((Nk, d), 123), _rand((Nk, d), 124)
+    q = _rand((Nq, d), 125)
+    for off in (-8, -3, 0, 4, 11, 14):
+        for causal, window in MASKS:
+            O, lse = o.attention_forward_offset(np.zeros((Nq, d)), k, v, off, None, causal, window)
+            ok = np.zeros((Nq, Nk), dtype=bool)
+            for i in range(Nq):
+                p = off + i
+                js = [j for j in range(Nk)
+                      if (not causal or j <= p) and (window <= 0 or j > p - window)]
+                ok[i, js] = True
+                if js:
+                    assert np.abs(O[i] - v[js].mean(axis=0)).max() < 1e-14, (off, causal, window, i)
+                    assert abs(lse[i] - math.log(len(js))) < 1e-14, (off, causal, window, i)
+                else:
+                    assert np.all(O[i] == 0.0) and lse[i] == -np.inf, (off, causal, window, i)
+            live = ok.any(axis=1)
+            if not live.any():
+                continue
+            O, _ = o.attention_forward_offset(q, k, v, off, 0.6, causal, window)
+            ref = F.scaled_dot_product_attention(
+                torch.from_numpy(q[live]), torch.from_numpy(k), torch.from_numpy(v),
+                attn_mask=torch.from_numpy(ok[live]), scale=0.6).numpy()
+            assert np.abs(O[live] - ref).max() < 1e-12, (off, causal, window)
+
+
 ALL_PINS = [
     pin_worked_example_tiled,
     pin_worked_example_naive,
@@ -335,4 +391,6 @@ ALL_PINS = [
     pin_paged_decode,
     pin_merge,
     pin_rows_subset,
+    pin_offset_shards,
+    pin_offset_closed_form,
 ]

@@ -143,6 +143,18 @@ def _paged_blocks_reversed(q, kpool, vpool, block_table, seqlens, scale=None):
             vc[b, :, t * bs:(t + 1) * bs] = vpool[table[b, nb - 1 - t]]
     return _real_decode(q, kc, vc, n, scale)
 
+def _offset_factory(mistake):
+    def fwd(q, k, v, q_offset, scale=None, causal=False, window=0):
+        n_q = np.asarray(q).shape[-2]
+        if mistake == "sign":
+            q_pos = np.arange(n_q) - q_offset       # key shard taken as ahead of the queries
+        else:
+            q_pos = np.arange(n_q)                  # offset ignored: every shard seen as the diagonal
+        P, lse = om.attention_probabilities(q, k, scale, causal, window, q_pos=q_pos)
+        return P @ np.asarray(v, dtype=np.float64), lse
+    return fwd
+
+
 MUTANTS = {
     "window_off_by_one": ("allowed_mask", _mask_window_off_by_one),
     "causal_drops_diagonal": ("allowed_mask", _mask_strict_causal),
@@ -156,6 +168,8 @@ MUTANTS = {
     "decode_reads_past_seqlen": ("decode_forward", _decode_reads_one_extra),
     "merge_unweighted": ("merge_partials", _merge_unweighted),
     "paged_blocks_reversed": ("decode_paged_forward", _paged_blocks_reversed),
+    "offset_sign_flipped": ("attention_forward_offset", _offset_factory("sign")),
+    "offset_ignored": ("attention_forward_offset", _offset_factory("ignored")),
 }
 
 
