@@ -289,6 +289,9 @@ def make_step(w, dev):
         return (step, e2e, units, "GB/s", "decode GB/s", 2, "decode_split_kernel",
                 ["decode.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
+    if w.kind == "context_parallel":
+        return _context_parallel_step(w, dev, fa)
+
     with_bwd = w.kind == "forward_backward"
     ins = workloads.workload_inputs(w, device=dev)
     q, k, v = ins[:3]
@@ -325,6 +328,67 @@ def make_step(w, dev):
     return (step, e2e, flops / 1e12, "TFLOP/s", metric, 4 if with_bwd else 1,
             "bwd_main_kernel" if with_bwd else "fwd_tc_kernel",
             ["bwd.cu" if with_bwd else "fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
+
+
+def context_parallel_plan(w):
+    """Per rank of the ring: the key shards it computes (visible ones), in ring order."""
+    from tiled_exact_attention_forward_b200 import context_parallel as cp
+
+    Ns = w.N // w.shards
+    return Ns, [[st for st in cp.ring_schedule(r, w.shards, Ns, w.causal, w.window) if st.visible]
+                for r in range(w.shards)]
+
+
+def context_parallel_emulated(w, dev, fa):
+    """All ranks of the ring on one device: each rank's sequence shard of q, k, v,
+    the key-shard partials it computes and the merge.  The exchange itself (NCCL
+    send/receive between GPUs) is not part of it: one GPU has no peer.
+    Returns (step, shards (q, k, v lists), results (o, lse lists), launches)."""
+    q, k, v = workloads.workload_inputs(w, device=dev)
+    Ns, plans = context_parallel_plan(w)
+    cut = [[t[:, :, r * Ns:(r + 1) * Ns].contiguous() for r in range(w.shards)] for t in (q, k, v)]
+    del q, k, v
+    qs, ks, vs = cut
+    o_parts = [torch.empty((len(p), w.B, w.H, Ns, w.d), dtype=w.dtype, device=dev) for p in plans]
+    l_parts = [torch.empty((len(p), w.B, w.H, Ns), dtype=torch.float32, device=dev) for p in plans]
+    merged = [len(p) > 1 for p in plans]
+    outs = [torch.empty_like(qs[r]) if merged[r] else o_parts[r][0] for r in range(w.shards)]
+    lses = [torch.empty((w.B, w.H, Ns), dtype=torch.float32, device=dev) if merged[r] else l_parts[r][0]
+            for r in range(w.shards)]
+
+    def step():
+        for r, plan in enumerate(plans):
+            for i, st in enumerate(plan):
+                fa.forward_offset(qs[r], ks[st.shard], vs[st.shard], st.q_offset, w.causal, w.window,
+                                  w.scale, out=o_parts[r][i], lse=l_parts[r][i])
+            if merged[r]:
+                fa.merge(o_parts[r], l_parts[r], out=outs[r], lse=lses[r])
+
+    launches = sum(len(p) for p in plans) + sum(merged)
+    return step, (qs, ks, vs), (outs, lses), launches
+
+
+def _context_parallel_step(w, dev, fa):
+    step, (qs, ks, vs), (outs, lses), launches = context_parallel_emulated(w, dev, fa)
+    host_in = [t.cpu().pin_memory() for t in qs + ks + vs]
+    dev_in = qs + ks + vs
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs + lses]
+    dev_out = outs + lses
+
+    # End to end: every rank's shards go up from pinned host memory, the ring steps
+    # run, and every rank's output rows and lse come back.
+    def e2e():
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in zip(host_out, dev_out):
+            h_.copy_(d_, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    return (step, e2e, forward_flops(w) / 1e12, "TFLOP/s", "attention TFLOP/s (fwd, unmasked FLOPs)",
+            launches, "fwd_tc_kernel", ["fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
 def max_over_ranks(values, device=None):
@@ -411,7 +475,9 @@ def run_gpu(args, rank, world, local_rank):
                    "window": w.window, "global_batch": w.B * world, "seq_len": w.N,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
-                   **({"block_size": w.block_size} if w.block_size else {})},
+                   **({"block_size": w.block_size} if w.block_size else {}),
+                   **({"shards": w.shards, "ring": "every rank's steps on one GPU, exchange not timed"}
+                      if w.shards else {})},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches * args.steps,

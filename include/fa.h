@@ -16,6 +16,9 @@
  *     Extending It (paged KV-cache integration, read as a block pool).
  *   - "Build a FlashAttention Kernel with Online Softmax and KV Cache in Pure
  *     Python": Step 4 (single-query decode against a key/value cache).
+ *   - Both pure-Python pages' "Extending It" roadmaps (attention split across
+ *     devices, each holding part of the key/value space): the per-shard
+ *     forward fa_forward_offset and the partial-result merge fa_merge.
  *
  * Conventions shared by every entry point
  *   - Layout: Q, K, V, O, dO, dQ, dK, dV are contiguous row-major
@@ -92,6 +95,46 @@ typedef enum {
 FA_API fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d, float scale, int causal, int window,
                      fa_dtype dtype, void* stream);
+
+/*
+ * One key shard's forward, for context-parallel attention: queries against a
+ * contiguous run of keys that starts `q_offset` positions before query row 0.
+ * Both pure-Python kernel pages' "Extending It" roadmaps (the attention matrix
+ * split across devices; each worker holds part of the key/value space).
+ *
+ *   q, o    : [B][H][Nq][d]; k, v: [B][H][Nk][d] (FA_BF16 or FA_FP16,
+ *             d = 128), 16-byte aligned.  lse: [B][H][Nq] float32 or NULL.
+ *   q_offset: query row i sits at position i + q_offset of the key sequence,
+ *             so the mask is (causal == 0 || j <= i + q_offset) &&
+ *             (window <= 0 || j > i + q_offset - window), j in [0, Nk).  0
+ *             with Nq == Nk is fa_forward.  |q_offset|, Nq, Nk and window must
+ *             not exceed 2^29 (FA_ERR_INVALID otherwise).
+ * O and lse are the softmax over this shard's keys only; a row that sees none
+ * of them gets O = 0 and lse = -inf (query tiles with no visible key run no
+ * MMA at all).  fa_merge combines the shards' results into the full
+ * attention.
+ */
+FA_API fa_status fa_forward_offset(const void* q, const void* k, const void* v, void* o, float* lse,
+                                   int B, int H, int Nq, int Nk, int q_offset, int d, float scale,
+                                   int causal, int window, fa_dtype dtype, void* stream);
+
+/*
+ * Merge of S partial results over disjoint key sets.  "Building Flash
+ * Attention from Scratch in Pure NumPy", architecture overview (the merge
+ * identity for two partial softmaxes, restated for S parts):
+ *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+ *
+ *   o_parts   : [S][B][H][N][d] normalised partial outputs (FA_BF16 or
+ *               FA_FP16, d = 64 or 128), 16-byte aligned.
+ *   lse_parts : [S][B][H][N] float32; -inf marks a part with no visible key
+ *               for that row (its O is not read).
+ *   o         : [B][H][N][d] output; lse: [B][H][N] float32 output or NULL.
+ *   S         : 1 .. 65536.
+ * A row whose parts are all empty gets O = 0 and lse = -inf; a NaN lse in any
+ * part makes the row NaN.
+ */
+FA_API fa_status fa_merge(const void* o_parts, const float* lse_parts, int S, void* o, float* lse,
+                          int B, int H, int N, int d, fa_dtype dtype, void* stream);
 
 /*
  * Bytes of device workspace fa_decode needs for these sizes (a multiple of

@@ -37,7 +37,8 @@ def test_status_strings_and_version(lib):
     for code in range(5):
         assert lib.fa_status_string(code).startswith(b"FA_")
     assert lib.fa_status_string(99) == b"unknown fa_status"
-    assert lib.fa_version() == 101  # 1.01: fa_decode_paged and FA_FP16 added to 1.00
+    # 1.02: fa_forward_offset and fa_merge added to 1.01 (fa_decode_paged, FA_FP16).
+    assert lib.fa_version() == 102
 
 
 P = ctypes.c_void_p
@@ -63,6 +64,42 @@ def test_forward_rejects_bad_arguments(lib):
     assert fwd(lib, d=64) == fa.FA_ERR_UNSUPPORTED          # bf16 needs d = 128
     assert fwd(lib, d=96, dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
     assert fwd(lib, dtype=7) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_forward_offset_rejects_bad_arguments(lib):
+    def fo(q=GOOD, lse=None, Nq=128, Nk=200, off=0, d=128, causal=1, window=0, dtype=fa.FA_BF16):
+        return lib.fa_forward_offset(q, GOOD, GOOD, GOOD, lse, 1, 2, Nq, Nk, off, d, 0.0, causal,
+                                     window, dtype, None)
+
+    assert fo(q=None) == fa.FA_ERR_INVALID
+    assert fo(Nq=0) == fa.FA_ERR_INVALID
+    assert fo(Nk=0) == fa.FA_ERR_INVALID
+    assert fo(Nk=(1 << 29) + 1) == fa.FA_ERR_INVALID
+    assert fo(off=(1 << 29) + 1) == fa.FA_ERR_INVALID
+    assert fo(off=-(1 << 29) - 1) == fa.FA_ERR_INVALID
+    assert fo(window=(1 << 29) + 1) == fa.FA_ERR_INVALID
+    assert fo(window=-1) == fa.FA_ERR_INVALID
+    assert fo(causal=3) == fa.FA_ERR_INVALID
+    assert fo(q=MISALIGNED) == fa.FA_ERR_INVALID
+    assert fo(lse=P(0x100001)) == fa.FA_ERR_INVALID
+    assert fo(d=64) == fa.FA_ERR_UNSUPPORTED
+    assert fo(dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_merge_rejects_bad_arguments(lib):
+    def mg(parts=GOOD, lse_parts=GOOD, S=3, o=GOOD, N=100, d=128, dtype=fa.FA_BF16):
+        return lib.fa_merge(parts, lse_parts, S, o, None, 2, 3, N, d, dtype, None)
+
+    assert mg(parts=None) == fa.FA_ERR_INVALID
+    assert mg(lse_parts=None) == fa.FA_ERR_INVALID
+    assert mg(o=None) == fa.FA_ERR_INVALID
+    assert mg(S=0) == fa.FA_ERR_INVALID
+    assert mg(S=(1 << 16) + 1) == fa.FA_ERR_INVALID
+    assert mg(N=0) == fa.FA_ERR_INVALID
+    assert mg(parts=MISALIGNED) == fa.FA_ERR_INVALID
+    assert mg(lse_parts=P(0x100002)) == fa.FA_ERR_INVALID
+    assert mg(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert mg(dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments(lib):

@@ -12,10 +12,15 @@ Functions (names follow the C ABI):
     decode_paged(q, kpool, vpool, block_table, seqlens)          -> (o, lse)
     backward(q, k, v, o, dout, lse, causal=False, window=0,
              scale=None)                                         -> (dq, dk, dv)
+    forward_offset(q, k, v, q_offset, causal=False, window=0)   -> (o, lse)
+    merge(o_parts, lse_parts)                                    -> (o, lse)
     forward_host(...)  -- forward on pinned host tensors (copies in and out)
     forward_backward_host(...)  -- forward and backward on pinned host tensors
     attention(q, k, v, causal=False, window=0, scale=None)      -> o, differentiable
     device_status()    -- FA_OK or the first recorded device-side timeout
+
+The ring (context-parallel) forward over torch.distributed ranks sits in
+``context_parallel``; its compute is ``forward_offset`` and ``merge``.
 """
 from __future__ import annotations
 
@@ -32,6 +37,8 @@ FA_BF16, FA_FP32, FA_FP16 = 0, 1, 2
 
 EXPORTED_SYMBOLS = (
     "fa_forward",
+    "fa_forward_offset",
+    "fa_merge",
     "fa_decode_workspace_size",
     "fa_decode",
     "fa_decode_noalloc",
@@ -69,6 +76,10 @@ def _lib() -> ctypes.CDLL:
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_forward.argtypes = [P, P, P, P, P, I, I, I, I, F, I, I, I, P]
     lib.fa_forward.restype = I
+    lib.fa_forward_offset.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P]
+    lib.fa_forward_offset.restype = I
+    lib.fa_merge.argtypes = [P, P, I, P, P, I, I, I, I, I, P]
+    lib.fa_merge.restype = I
     lib.fa_decode_workspace_size.argtypes = [I, I, I, I]
     lib.fa_decode_workspace_size.restype = Z
     lib.fa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, F, I, P, Z, P]
@@ -152,6 +163,53 @@ def forward(q, k, v, causal: bool = False, window: int = 0, scale=None, out=None
                            _scale_arg(scale), int(bool(causal)), int(window),
                            _dtype_code(q.dtype), _stream(q.device))
     _check(st, "fa_forward")
+    return o, lse
+
+
+def forward_offset(q, k, v, q_offset: int, causal: bool = False, window: int = 0, scale=None,
+                   out=None, lse=None):
+    """One key shard's partial forward (context parallelism).
+
+    q: [B, H, Nq, d]; k, v: [B, H, Nk, d] (bf16 or fp16, d = 128), contiguous CUDA
+    tensors.  Query row i sits at position i + q_offset of the key sequence; the
+    causal and window masks are taken at those positions.  Returns (o, lse): the
+    softmax over these keys only, o like q, lse [B, H, Nq] (-inf, with o = 0, for
+    a row that sees none of the keys).
+    """
+    _need_cuda(q, k, v)
+    B, H, Nq, d = q.shape
+    if k.dim() != 4 or k.shape[:2] != (B, H) or k.shape[3] != d or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H and d")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype")
+    Nk = k.shape[2]
+    o = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    st = _lib().fa_forward_offset(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk,
+                                  int(q_offset), d, _scale_arg(scale), int(bool(causal)), int(window),
+                                  _dtype_code(q.dtype), _stream(q.device))
+    _check(st, "fa_forward_offset")
+    return o, lse
+
+
+def merge(o_parts, lse_parts, out=None, lse=None):
+    """Combine S partial results over disjoint key sets into the full attention.
+
+    o_parts: [S, B, H, N, d] (bf16 or fp16, d in {64, 128}); lse_parts:
+    [S, B, H, N] float32 (-inf marks a part that saw no key for that row).
+    Returns (o [B, H, N, d], lse [B, H, N]).
+    """
+    _need_cuda(o_parts, lse_parts)
+    S, B, H, N, d = o_parts.shape
+    if lse_parts.shape != (S, B, H, N) or lse_parts.dtype != torch.float32:
+        raise ValueError("lse_parts must be float32 [S, B, H, N] matching o_parts")
+    o = torch.empty(o_parts.shape[1:], dtype=o_parts.dtype, device=o_parts.device) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=o_parts.device)
+    st = _lib().fa_merge(_ptr(o_parts), _ptr(lse_parts), S, _ptr(o), _ptr(lse), B, H, N, d,
+                         _dtype_code(o_parts.dtype), _stream(o_parts.device))
+    _check(st, "fa_merge")
     return o, lse
 
 

@@ -32,7 +32,7 @@ bool sizes_ok(long long B, long long H, long long N) {
 
 extern "C" {
 
-int fa_version(void) { return 101; }
+int fa_version(void) { return 102; }
 
 const char* fa_status_string(fa_status s) {
   switch (s) {
@@ -55,6 +55,7 @@ fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float
   fa::FwdArgs a{};
   a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
   a.B = B; a.H = H; a.N = N; a.d = d;
+  a.Nk = N; a.q_off = 0;
   a.causal = causal; a.window = window;
   a.scale = resolve_scale(scale, d);
   a.scale_log2 = a.scale * kLog2e;
@@ -69,6 +70,45 @@ fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float
     return from_cuda(fa::launch_fwd_f32(a, st));
   }
   return FA_ERR_UNSUPPORTED;
+}
+
+fa_status fa_forward_offset(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                            int H, int Nq, int Nk, int q_offset, int d, float scale, int causal,
+                            int window, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID;
+  // Positions (row + q_offset, minus window, minus a key index) must stay inside int.
+  constexpr int kLimit = 1 << 29;
+  if (!sizes_ok(B, H, Nq) || Nk < 1 || Nq > kLimit || Nk > kLimit || q_offset > kLimit ||
+      q_offset < -kLimit || window < 0 || window > kLimit || (causal != 0 && causal != 1))
+    return FA_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID;
+  if ((dtype != FA_BF16 && dtype != FA_FP16) || d != 128) return FA_ERR_UNSUPPORTED;
+  fa::FwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.o = o; a.lse = lse;
+  a.B = B; a.H = H; a.N = Nq; a.d = d;
+  a.Nk = Nk; a.q_off = q_offset;
+  a.causal = causal; a.window = window;
+  a.scale = resolve_scale(scale, d);
+  a.scale_log2 = a.scale * kLog2e;
+  a.f16 = dtype == FA_FP16;
+  return from_cuda(fa::launch_fwd_tc(a, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_merge(const void* o_parts, const float* lse_parts, int S, void* o, float* lse, int B,
+                   int H, int N, int d, fa_dtype dtype, void* stream) {
+  if (!o_parts || !lse_parts || !o) return FA_ERR_INVALID;
+  if (S < 1 || S > (1 << 16) || !sizes_ok(B, H, N)) return FA_ERR_INVALID;
+  if (!aligned(o_parts, 16) || !aligned(o, 16) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
+    return FA_ERR_INVALID;
+  if ((dtype != FA_BF16 && dtype != FA_FP16) || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  fa::MergeArgs a{};
+  a.o_parts = o_parts; a.lse_parts = lse_parts; a.o = o; a.lse = lse;
+  a.rows = static_cast<long long>(B) * H * N;
+  a.S = S; a.d = d;
+  a.f16 = dtype == FA_FP16;
+  return from_cuda(fa::launch_merge(a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t fa_decode_workspace_size(int B, int H, int cap, int d) {

@@ -92,21 +92,39 @@ struct Smem {
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
-// Key-tile range [lo, hi) a query tile starting at row r0 must visit.
-__device__ __forceinline__ void key_tile_range(int r0, int n, int causal, int window, int& lo,
-                                               int& hi) {
-  const int rlast = min(r0 + BM - 1, n - 1);
-  hi = causal ? (rlast / BN + 1) : (n + BN - 1) / BN;
-  const int first_key = window > 0 ? r0 - window + 1 : 0;
+// Positions: query row i sits at position i + q_off of the key sequence (q_off = 0
+// and Nk = N for self-attention; a context-parallel shard passes the distance
+// between its query rows and the key shard).  Key j of [0, Nk) is visible to row i
+// iff (!causal || j <= i + q_off) && (window == 0 || j > i + q_off - window).
+
+// The sizes and mask of one launch, held in registers (a reference to the kernel
+// parameter itself would force a copy of it to local memory).
+struct Geom {
+  int N, Nk, q_off, causal, window;
+};
+
+// Key-tile range [lo, hi) a query tile starting at row r0 must visit (empty when
+// no row of the tile sees any key).
+template <bool OFFSET>
+__device__ __forceinline__ void key_tile_range(int r0, const Geom& a, int& lo, int& hi) {
+  const int rlast = min(r0 + BM - 1, a.N - 1);
+  const int p0 = r0 + a.q_off, p1 = rlast + a.q_off;  // positions of the first and last row
+  const int nkt = (a.Nk + BN - 1) / BN;
+  if (!OFFSET)  // rlast < N = Nk: the causal bound needs no clamp
+    hi = a.causal ? (rlast / BN + 1) : nkt;
+  else
+    hi = a.causal ? (p1 < 0 ? 0 : min(nkt, p1 / BN + 1)) : nkt;
+  const int first_key = a.window > 0 ? p0 - a.window + 1 : 0;
   lo = first_key > 0 ? first_key / BN : 0;
   if (lo > hi) lo = hi;
 }
 
 // Does key tile j need the per-element mask for rows r0..r0+BM-1?
-__device__ __forceinline__ bool tile_needs_mask(int j, int r0, int n, int causal, int window) {
+__device__ __forceinline__ bool tile_needs_mask(int j, int r0, const Geom& a) {
   const int k0 = j * BN, k1 = j * BN + BN - 1;
-  const int rlast = min(r0 + BM - 1, n - 1);
-  return (k1 >= n) || (causal && k1 > r0) || (window > 0 && k0 <= rlast - window);
+  const int rlast = min(r0 + BM - 1, a.N - 1);
+  const int p0 = r0 + a.q_off, p1 = rlast + a.q_off;
+  return (k1 >= a.Nk) || (a.causal && k1 > p0) || (a.window > 0 && k0 <= p1 - a.window);
 }
 
 // 128-byte-swizzled shared-memory matrix descriptor as two 32-bit words: the
@@ -149,16 +167,23 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
 }
 
 // One unit of work: two 128-row query tiles (rows [256p, 256p + 256)) of one
-// (batch, head), with the key-tile range each of them must visit.
+// (batch, head), with the key-tile range each of them must visit.  A tile that
+// exists but sees no key (possible only with a query offset) is inactive: no Q
+// load, no MMA; its softmax warps write O = 0 and lse = -inf directly.
 struct Item {
   int bh;
   int r0[2];
   int lo_t[2], hi_t[2];
-  int lo, hi;
-  bool has1;
+  int lo, hi;  // union of the active tiles' ranges (empty if none is active)
+  bool has1;   // tile 1 exists (rows below N)
+  __device__ __forceinline__ bool active(int t) const { return lo_t[t] < hi_t[t]; }
 };
 
-__device__ __forceinline__ Item make_item(int lin, int BH, int n, int num_pairs, int causal, int window) {
+// OFFSET: the launch may have a query offset or Nk != N (context-parallel shards),
+// so tiles can be inactive.  Self-attention (OFFSET false) has every existing tile
+// active: its diagonal key tile is always visible.
+template <bool OFFSET>
+__device__ __forceinline__ Item make_item(int lin, int BH, int num_pairs, const Geom& a) {
   Item it;
   // Heaviest work first: with a causal mask the last query tiles see the most keys.
   const int pair = num_pairs - 1 - lin / BH;
@@ -167,15 +192,24 @@ __device__ __forceinline__ Item make_item(int lin, int BH, int n, int num_pairs,
   it.r0[1] = it.r0[0] + BM;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    if (it.r0[t] < n) {
-      key_tile_range(it.r0[t], n, causal, window, it.lo_t[t], it.hi_t[t]);
+    if (it.r0[t] < a.N) {
+      key_tile_range<OFFSET>(it.r0[t], a, it.lo_t[t], it.hi_t[t]);
     } else {
       it.lo_t[t] = it.hi_t[t] = 0;
     }
   }
-  it.has1 = it.r0[1] < n;
-  it.lo = it.has1 ? min(it.lo_t[0], it.lo_t[1]) : it.lo_t[0];
-  it.hi = it.has1 ? max(it.hi_t[0], it.hi_t[1]) : it.hi_t[0];
+  it.has1 = it.r0[1] < a.N;
+  if (!OFFSET) {
+    it.lo = it.has1 ? min(it.lo_t[0], it.lo_t[1]) : it.lo_t[0];
+    it.hi = it.has1 ? max(it.hi_t[0], it.hi_t[1]) : it.hi_t[0];
+  } else if (it.active(0) && it.active(1)) {
+    it.lo = min(it.lo_t[0], it.lo_t[1]);
+    it.hi = max(it.hi_t[0], it.hi_t[1]);
+  } else {
+    const int t = it.active(1) ? 1 : 0;
+    it.lo = it.active(t) ? it.lo_t[t] : 0;
+    it.hi = it.active(t) ? it.hi_t[t] : 0;
+  }
   return it;
 }
 
@@ -188,8 +222,8 @@ __device__ __forceinline__ int item_of(int k, int total) {
   return lin < total ? lin : -1;
 }
 
-// T: the 16-bit type of Q, K, V, P and O (Bf16 or F16).
-template <class T>
+// T: the 16-bit type of Q, K, V, P and O (Bf16 or F16).  OFFSET: see make_item.
+template <class T, bool OFFSET>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, FwdArgs args) {
@@ -202,6 +236,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n = args.N;
   const int num_pairs = (n + 2 * BM - 1) / (2 * BM);
   const int total = num_pairs * BH;
+  const Geom geo{args.N, OFFSET ? args.Nk : args.N, OFFSET ? args.q_off : 0, args.causal, args.window};
+  // Is tile t of an item to be computed?  (Without an offset: whenever it exists.)
+  auto active = [](const Item& it, int t) { return OFFSET ? it.active(t) : (t == 0 || it.has1); };
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -245,8 +282,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int lin = item_of(k, total);
         if (lin < 0) break;
-        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
-        for (int t = 0; t < (it.has1 ? 2 : 1) && ok; ++t) {
+        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!active(it, t)) continue;
           if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
           if (!ok) break;
           const uint32_t bar = smem_u32(&sm.q_full[t]);
@@ -267,7 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int lin = item_of(k, total);
         if (lin < 0) break;
-        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
         for (int idx = 0; ok && idx < 2 * (it.hi - it.lo); ++idx, ++kvi) {
           const int s = kvi % NS;
           if (kvi >= NS) ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((kvi / NS) - 1) & 1, abort_flag);
@@ -319,7 +357,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int k = 0; ok; ++k) {
         const int lin = item_of(k, total);
         if (lin < 0) break;
-        const Item it = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
         auto act = [&](int t, int j) { return j >= it.lo_t[t] && j < it.hi_t[t]; };
         // PV_t(j): the first one of an item overwrites O_t, so the previous item's
         // epilogue must have read it out; the last one publishes O_t.
@@ -337,7 +375,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           return true;
         };
-        if (it.hi <= it.lo) break;
+        if (it.hi <= it.lo) {  // no active tile: nothing to issue
+          if (OFFSET) continue;
+          break;
+        }
         // Prologue: S_t(lo) for both tiles (S_0(lo) may already be in flight).
         ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi)]), parity_of(kvi), abort_flag);
         if (!ok) break;
@@ -382,8 +423,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (j == it.hi - 2 && it.has1 && !act(0, j + 1)) {
             const int lin2 = item_of(k + 1, total);
             if (lin2 >= 0) {
-              const Item nx = make_item(lin2, BH, n, num_pairs, args.causal, args.window);
-              if (nx.hi > nx.lo && nx.lo_t[0] == nx.lo) {
+              const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
+              if (active(nx, 0) && nx.lo_t[0] == nx.lo) {
                 ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi + 1)]), parity_of(kvi + 1), abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -422,10 +463,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int k = 0; ok; ++k) {
       const int lin = item_of(k, total);
       if (lin < 0) break;
-      const Item item = make_item(lin, BH, n, num_pairs, args.causal, args.window);
+      const Item item = make_item<OFFSET>(lin, BH, num_pairs, geo);
       if (t == 1 && !item.has1) continue;
       const int r0 = item.r0[t];
       const int row_g = r0 + row;
+      if (OFFSET && !item.active(t)) {
+        // No row of this tile sees a key: O = 0, lse = -inf.
+        if (row_g < n) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.o) +
+                                                (static_cast<size_t>(item.bh) * n + row_g) * D + 64 * hc);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+          if (hc == 0 && args.lse != nullptr) args.lse[static_cast<size_t>(item.bh) * n + row_g] = -INFINITY;
+        }
+        continue;
+      }
+      const int row_p = row_g + geo.q_off;  // the row's position in the key sequence
       float m = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
       bool nan_row = false;
       for (int j = item.lo_t[t]; j < item.hi_t[t]; ++j, ++ns) {
@@ -435,13 +488,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         FA_TMEM_LD32(tS + 0, (s + 0));
         FA_TMEM_LD32(tS + 32, (s + 32));
         tmem_ld_wait();
-        const bool masked = tile_needs_mask(j, r0, n, args.causal, args.window);
+        const bool masked = tile_needs_mask(j, r0, geo);
         if (masked) {
           // Visible keys of this row form one interval; columns of this half are 64h + c.
           const int base = j * BN + 64 * hc;
-          int c_hi = min(64, n - base);
-          if (args.causal) c_hi = min(c_hi, row_g - base + 1);
-          const int c_lo = args.window > 0 ? max(0, row_g - args.window + 1 - base) : 0;
+          int c_hi = min(64, geo.Nk - base);
+          if (args.causal) c_hi = min(c_hi, row_p - base + 1);
+          const int c_lo = args.window > 0 ? max(0, row_p - args.window + 1 - base) : 0;
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
@@ -551,6 +604,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       float lt = l + sm.xsum[t][hc ^ 1][row];
       // The sums may be read again only after the next item's first exchange barrier.
+      // A row whose max is still -inf saw no key: its sum is only the cubic's floor
+      // for masked scores (< 1e-38 each), not probability mass.
+      if (OFFSET && m == -INFINITY) lt = 0.f;
       if (nan_row) lt = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
       const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
       if (row_g < n) {
@@ -588,10 +644,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
   const long long heads = static_cast<long long>(a.B) * a.H;
   if (!make_tmap_half_rows(&tq, a.q, D, a.N, heads, BM, a.f16) ||
-      !make_tmap_half_rows(&tk, a.k, D, a.N, heads, BN, a.f16) ||
-      !make_tmap_half_rows(&tv, a.v, D, a.N, heads, BN, a.f16))
+      !make_tmap_half_rows(&tk, a.k, D, a.Nk, heads, BN, a.f16) ||
+      !make_tmap_half_rows(&tv, a.v, D, a.Nk, heads, BN, a.f16))
     return cudaErrorInvalidValue;
-  auto kernel = a.f16 ? fwd_tc_kernel<F16> : fwd_tc_kernel<Bf16>;
+  const bool offset = a.q_off != 0 || a.Nk != a.N;
+  auto kernel = offset ? (a.f16 ? fwd_tc_kernel<F16, true> : fwd_tc_kernel<Bf16, true>)
+                       : (a.f16 ? fwd_tc_kernel<F16, false> : fwd_tc_kernel<Bf16, false>);
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>((a.N + 2 * BM - 1) / (2 * BM)) * heads;

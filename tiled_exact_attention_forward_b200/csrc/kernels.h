@@ -13,11 +13,13 @@ struct FwdArgs {
   const void* v;
   void* o;
   float* lse;  // may be null
-  int B, H, N, d;
+  int B, H, N, d;     // N: query rows per head
   int causal, window;
   float scale;       // natural units
   float scale_log2;  // scale * log2(e)
   int f16;           // 16-bit inputs/outputs are f16 (else bf16)
+  int Nk;            // key rows per head (N for self-attention)
+  int q_off;         // position of query row 0 in the key sequence (0 for self-attention)
 };
 
 struct DecodeArgs {
@@ -62,6 +64,17 @@ struct BwdArgs {
   int f16;          // 16-bit tensors are f16 (else bf16)
 };
 
+// Merge of partial results over disjoint key sets (context parallelism).
+struct MergeArgs {
+  const void* o_parts;     // [S][rows][d] 16-bit, each part normalised
+  const float* lse_parts;  // [S][rows]; -inf marks a part that saw no key
+  void* o;                 // [rows][d] 16-bit
+  float* lse;              // [rows], may be null
+  long long rows;          // B * H * N
+  int S, d;
+  int f16;
+};
+
 // Decode: keys per split chunk (one CTA each).
 constexpr int kDecodeChunk = 512;
 
@@ -85,6 +98,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, cudaStream_t stream);
 
 }  // namespace fa

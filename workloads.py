@@ -30,7 +30,7 @@ class Workload:
     """One named attention workload (shapes, masks, dtype, seed)."""
 
     name: str
-    kind: str            # "forward", "decode" or "forward_backward"
+    kind: str            # "forward", "decode", "paged_decode", "forward_backward" or "context_parallel"
     B: int
     H: int
     N: int               # sequence length (decode: cache capacity)
@@ -42,6 +42,7 @@ class Workload:
     seqlen_lo: int = 0   # decode only: per-sequence cache length range
     seqlen_hi: int = 0
     block_size: int = 0  # paged decode only: rows per cache block
+    shards: int = 0      # context parallel only: sequence shards (ranks of the ring)
     notes: str = field(default="", compare=False)
 
     @property
@@ -70,6 +71,10 @@ WORKLOADS = {
                  seqlen_lo=512, seqlen_hi=8192, block_size=16,
                  notes="single-token decode against a paged cache: 16-row blocks, "
                        "shuffled in one pool, the lengths of kv_cache_decode"),
+        Workload("context_parallel_causal", "context_parallel", 1, 32, 16384, 128, BF16, 5,
+                 causal=True, shards=4,
+                 notes="causal forward of a 16K context cut into 4 sequence shards: every "
+                       "rank's ring steps (key-shard partials, then the merge) run on one GPU"),
     ]
 }
 
