@@ -143,3 +143,12 @@ def test_bench_plan_partitions_the_visible_pairs():
                 ok = oracle.allowed_mask(Ns, Ns, causal, window, q_pos=np.arange(Ns) + st.q_offset)
                 total += int(ok.sum())
         assert total == bench.allowed_pairs(96, causal, window), (causal, window)
+
+
+def test_ring_forward_checks_shapes_before_any_exchange():
+    q = torch.zeros((1, 2, 8, 4), dtype=torch.float64)
+    ring = cp.RingForward(_oracle_partial, _oracle_merge)
+    with pytest.raises(ValueError):
+        ring(q, q[:, :, :4], q)
+    with pytest.raises(ValueError):
+        ring(q, q.transpose(2, 3).contiguous().transpose(2, 3), q)

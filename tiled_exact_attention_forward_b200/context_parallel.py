@@ -83,6 +83,9 @@ class RingForward:
     def __call__(self, q, k, v, causal: bool = False, window: int = 0, scale=None):
         if q.shape != k.shape or q.shape != v.shape:
             raise ValueError("each rank holds equal-length shards: q, k, v of one shape [B, H, Ns, d]")
+        if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+            # Checked before the first exchange is posted: a peer may already be waiting on it.
+            raise ValueError("q, k, v must be contiguous")
         world = dist.get_world_size(self.group) if dist.is_initialized() else 1
         rank = dist.get_rank(self.group) if dist.is_initialized() else 0
         B, H, Ns, d = q.shape
