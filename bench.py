@@ -519,7 +519,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   "window": w.window},
+                   "window": w.window,
+                   **({"block_size": w.block_size} if w.block_size else {}),
+                   **({"shards": w.shards, "ring": "the oracle takes the whole sequence at once (same result)"}
+                      if w.shards else {})},
         "cpu_baseline": {"kind": "oracle", "value": value, "unit": unit, "cores": cpu_threads_used(),
                          "sample": samples[-1] if samples else ""},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
