@@ -227,8 +227,10 @@ def oracle_sample(w, budget_s=12.0):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def make_step(w, dev):
-    """Returns (step_fn, e2e_fn, units_per_step, unit, metric, launches_per_step, kernel, sources)."""
+def make_step(w, dev, rank=0, world=1):
+    """Returns (step_fn, e2e_fn, units_per_step, unit, metric, launches_per_step, kernel, sources).
+
+    units and launches are this rank's share: the whole job is world x units."""
     import tiled_exact_attention_forward_b200 as fa
 
     if w.kind == "paged_decode":
@@ -290,6 +292,8 @@ def make_step(w, dev):
                 ["decode.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
     if w.kind == "context_parallel":
+        if world > 1:
+            return _ring_step(w, dev, fa, rank, world)
         return _context_parallel_step(w, dev, fa)
 
     with_bwd = w.kind == "forward_backward"
@@ -391,6 +395,50 @@ def _context_parallel_step(w, dev, fa):
             launches, "fwd_tc_kernel", ["fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
+def _ring_step(w, dev, fa, rank, world):
+    """The context-parallel ring across the ranks of the job: the sequence is cut into
+    `world` shards, rank r holds shard r of q, k and v, and each step is one
+    context_parallel_forward (key-shard partials, NCCL exchange of the K/V shards
+    around the ring, merge).  Every rank draws the same seeded full inputs and keeps
+    its own shard.  The total work is the whole sequence's, whatever `world` is."""
+    from tiled_exact_attention_forward_b200 import context_parallel as cp
+
+    if w.N % world:
+        raise ValueError(f"{w.name}: N = {w.N} does not split into {world} equal shards")
+    Ns = w.N // world
+    q, k, v = workloads.workload_inputs(w, device=dev)
+    qs, ks, vs = (t[:, :, rank * Ns:(rank + 1) * Ns].contiguous() for t in (q, k, v))
+    del q, k, v
+    out = {}
+
+    def step():
+        out["o"], out["lse"] = cp.context_parallel_forward(qs, ks, vs, w.causal, w.window, w.scale)
+
+    host_in = [t.cpu().pin_memory() for t in (qs, ks, vs)]
+    step()
+    torch.cuda.synchronize(dev)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out["o"], out["lse"])]
+
+    # End to end: this rank's shards go up from pinned host memory, the ring runs, and
+    # its output rows and lse come back.
+    def e2e():
+        for d_, h_ in zip((qs, ks, vs), host_in):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in zip(host_out, (out["o"], out["lse"])):
+            h_.copy_(d_, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    plans = [[st for st in cp.ring_schedule(r, world, Ns, w.causal, w.window) if st.visible]
+             for r in range(world)]
+    # Launches of the whole job per step, shared evenly (the line reports world x this).
+    launches = (sum(len(p) for p in plans) + sum(len(p) > 1 for p in plans)) / world
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    return (step, e2e, forward_flops(w) / 1e12 / world, "TFLOP/s", "attention TFLOP/s (fwd, unmasked FLOPs)",
+            launches, "fwd_tc_kernel", ["fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
+
+
 def max_over_ranks(values, device=None):
     """Element-wise max of per-rank values (the slowest rank sets the time)."""
     import torch.distributed as tdist
@@ -427,7 +475,8 @@ def run_gpu(args, rank, world, local_rank):
 
     fa.library()
     w = resolve_workload(args)
-    (step, e2e, units, unit, metric, launches, kernel, sources, h2d, d2h) = make_step(w, dev)
+    (step, e2e, units, unit, metric, launches, kernel, sources, h2d, d2h) = make_step(w, dev, rank, world)
+    ring = w.kind == "context_parallel" and world > 1
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     dist = world > 1
@@ -469,18 +518,21 @@ def run_gpu(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms,
         "ms_per_step_spread": {"p50": float(np.median(times)), "min": float(np.min(times)),
                                "max": float(np.max(times))},
-        "higher_is_better": True, "scaling": "weak",
+        "higher_is_better": True, "scaling": "strong" if ring else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), workloads.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-                   "window": w.window, "global_batch": w.B * world, "seq_len": w.N,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "window": w.window, "global_batch": w.B if ring else w.B * world, "seq_len": w.N,
+                   "parallelism": (f"context-parallel ring x{world}" if ring else
+                                   f"replicas x{world}" if world > 1 else "single GPU"),
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
                    **({"block_size": w.block_size} if w.block_size else {}),
-                   **({"shards": w.shards, "ring": "every rank's steps on one GPU, exchange not timed"}
+                   **({"shards": world, "ring": "one shard per GPU, NCCL exchange inside the timed steps"}
+                      if ring else
+                      {"shards": w.shards, "ring": "every rank's steps on one GPU, exchange not timed"}
                       if w.shards else {})},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": int(round(launches * (world if ring else 1) * args.steps)),
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
