@@ -145,6 +145,16 @@ def test_python_binding_refuses_cpu_tensors():
         fa.forward(q, q, q)
 
 
+def test_shard_forward_and_merge_refuse_cpu_tensors():
+    import torch
+
+    q = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward_offset(q, q, q, 0)
+    with pytest.raises(ValueError):
+        fa.merge(q[None], torch.zeros(1, 1, 1, 8))
+
+
 def test_forward_host_checks_its_inputs_before_touching_the_device():
     import torch
 
