@@ -395,6 +395,17 @@ def _context_parallel_step(w, dev, fa):
             launches, "fwd_tc_kernel", ["fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
+def ring_launches_per_step(w, world: int) -> int:
+    """Kernel launches of the whole job per ring step: every rank's visible key-shard
+    partials plus one merge on each rank that has more than one partial."""
+    from tiled_exact_attention_forward_b200 import context_parallel as cp
+
+    Ns = w.N // world
+    plans = [[st for st in cp.ring_schedule(r, world, Ns, w.causal, w.window) if st.visible]
+             for r in range(world)]
+    return sum(len(p) for p in plans) + sum(len(p) > 1 for p in plans)
+
+
 def _ring_step(w, dev, fa, rank, world):
     """The context-parallel ring across the ranks of the job: the sequence is cut into
     `world` shards, rank r holds shard r of q, k and v, and each step is one
@@ -429,10 +440,8 @@ def _ring_step(w, dev, fa, rank, world):
             h_.copy_(d_, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
 
-    plans = [[st for st in cp.ring_schedule(r, world, Ns, w.causal, w.window) if st.visible]
-             for r in range(world)]
     # Launches of the whole job per step, shared evenly (the line reports world x this).
-    launches = (sum(len(p) for p in plans) + sum(len(p) > 1 for p in plans)) / world
+    launches = ring_launches_per_step(w, world) / world
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
     return (step, e2e, forward_flops(w) / 1e12 / world, "TFLOP/s", "attention TFLOP/s (fwd, unmasked FLOPs)",

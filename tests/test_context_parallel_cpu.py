@@ -152,3 +152,25 @@ def test_ring_forward_checks_shapes_before_any_exchange():
         ring(q, q[:, :, :4], q)
     with pytest.raises(ValueError):
         ring(q, q.transpose(2, 3).contiguous().transpose(2, 3), q)
+
+
+def test_bench_ring_accounting():
+    """With N GPUs the bench runs one shard per rank: the whole job's launches per
+    step are the visible partials plus the merges, and the emulated one-GPU plan
+    of the same shard count launches exactly as many kernels."""
+    import dataclasses
+
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+
+    w = workloads.WORKLOADS["context_parallel_causal"]
+    # Causal, 4 shards: partials 1 + 2 + 3 + 4, merges on ranks 1-3.
+    assert bench.ring_launches_per_step(w, 4) == 13
+    assert bench.ring_launches_per_step(w, 1) == 1
+    assert bench.ring_launches_per_step(w, 2) == 4
+    for world in (2, 4, 8):
+        ww = dataclasses.replace(w, shards=world)
+        _, plans = bench.context_parallel_plan(ww)
+        assert bench.ring_launches_per_step(w, world) == \
+            sum(len(p) for p in plans) + sum(len(p) > 1 for p in plans)
