@@ -73,6 +73,11 @@ def decode_bytes(w, seqlens) -> float:
     return rows * w.d * 2 * 2 + 2 * w.B * w.H * w.d * 2 + table  # K + V rows, q + o, table
 
 
+def dtype_name(dtype) -> str:
+    """The arithmetic input type of a workload as the bench line names it."""
+    return {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[dtype]
+
+
 # ----------------------------------------------------------------------------- measurement helpers
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -528,7 +533,7 @@ def run_gpu(args, rank, world, local_rank):
         "ms_per_step_spread": {"p50": float(np.median(times)), "min": float(np.min(times)),
                                "max": float(np.max(times))},
         "higher_is_better": True, "scaling": "strong" if ring else "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1), workloads.py)",
+        "vs_baseline": None, "dtype": dtype_name(w.dtype), "data": "synthetic (seeded N(0,1), workloads.py)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "window": w.window, "global_batch": w.B if ring else w.B * world, "seq_len": w.N,
                    "parallelism": (f"context-parallel ring x{world}" if ring else

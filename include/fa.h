@@ -204,15 +204,20 @@ FA_API fa_status fa_decode_paged(const void* q, const void* kpool, const void* v
  * counterpart: this exists for deployment, not for the method.  Same arguments,
  * layout and results as fa_decode, minus the workspace: the per-chunk
  * partials go to a fixed array of FA_DECODE_NOALLOC_SCRATCH_BYTES compiled into
- * the library, which every GPU that loads the library holds until the process
- * exits.  Serving runtimes that forbid allocation after start-up and plugin
- * interfaces that pass a kernel only its inputs and outputs are the intended
- * users.
+ * the library.  Serving runtimes that forbid allocation after start-up and
+ * plugin interfaces that pass a kernel only its inputs and outputs are the
+ * intended users.
  *   - Size limit: fa_decode_workspace_size(B, H, cap, d) must not exceed
  *     FA_DECODE_NOALLOC_SCRATCH_BYTES (for cap = 8192 that is B*H <= 1016);
  *     larger calls return FA_ERR_INVALID with nothing launched.
- *   - The first call on each device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *   - With lazy module loading (the CUDA 12 default) the array is reserved on
+ *     a device by the first call made there (at library load instead when
+ *     CUDA_MODULE_LOADING=EAGER) and held until the process exits.  That first
+ *     call can fail with FA_ERR_CUDA when the device has no memory left, so
+ *     make it at start-up, as a warm-up, and before any stream capture.
+ *   - Every call looks the array's address up in the current context (the
+ *     address is per context: a device reset or another context moves it);
+ *     once loaded, the lookup does not synchronise.
  *   - All calls share the array: calls whose kernels overlap on the GPU race.
  *     Nothing needs clearing between calls.
  *   - Calls no cudaMalloc/cudaFree and no allocating library routine.
@@ -267,6 +272,19 @@ FA_API fa_status fa_get_device_status(void* stream);
  * `stream` reports it and clears it.  The CUDA context stays usable.
  */
 FA_API fa_status fa_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/*
+ * Self-test of the exponential used inside the forward softmax: writes
+ * y[i] = exp2_poly(x[i]) for i < n, where exp2_poly is the device function
+ * that computes part of "Building Flash Attention from Scratch in Pure NumPy",
+ * Step 2's P = exp(S - m_new) (in base 2) on the FMA pipe: a Cody-Waite
+ * split x = j + f, j = round(x), and a cubic in f fitted for minimum relative
+ * error.  Stated behaviour: relative error <= 7.5e-5 for -125.5 <= x <= 0;
+ * a result below 2^-125 for x < -125.5 (inputs are clamped at -126.5).
+ *   x, y : DEVICE float32 arrays of n elements (n >= 1), 4-byte aligned.
+ * Returns FA_ERR_INVALID for a null or misaligned pointer or n < 1.
+ */
+FA_API fa_status fa_selftest_exp2_poly(const float* x, float* y, long long n, void* stream);
 
 /* Static, human-readable name of a status code. */
 FA_API const char* fa_status_string(fa_status status);

@@ -37,8 +37,9 @@ def test_status_strings_and_version(lib):
     for code in range(5):
         assert lib.fa_status_string(code).startswith(b"FA_")
     assert lib.fa_status_string(99) == b"unknown fa_status"
-    # 1.02: fa_forward_offset and fa_merge added to 1.01 (fa_decode_paged, FA_FP16).
-    assert lib.fa_version() == 102
+    # 1.03: fa_selftest_exp2_poly added to 1.02 (fa_forward_offset, fa_merge), which
+    # added to 1.01 (fa_decode_paged, FA_FP16).
+    assert lib.fa_version() == 103
 
 
 P = ctypes.c_void_p
@@ -189,3 +190,33 @@ def test_decode_paged_rejects_bad_arguments(lib):
     assert dec(num_blocks=0) == fa.FA_ERR_INVALID
     assert dec(max_blocks=0) == fa.FA_ERR_INVALID
     assert dec(d=64) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_decode_noalloc_rejects_sizes_beyond_its_array(lib):
+    # The size check runs before any CUDA call, so the pointers (never
+    # dereferenced) can be fake; on a machine with a GPU nothing is launched
+    # either, because the sizes are refused first.
+    limit = 8 << 20
+    B, H, cap, d = 64, 32, 8192, 128          # ~17 MB of partials
+    assert lib.fa_decode_workspace_size(B, H, cap, d) > limit
+    st = lib.fa_decode_noalloc(GOOD, GOOD, GOOD, GOOD, GOOD, None, B, H, cap, d, 0.0, fa.FA_BF16, None)
+    assert st == fa.FA_ERR_INVALID
+    assert lib.fa_decode_workspace_size(1016, 1, cap, d) <= limit < lib.fa_decode_workspace_size(1017, 1, cap, d)
+    st = lib.fa_decode_noalloc(GOOD, GOOD, GOOD, GOOD, GOOD, None, 1017, 1, cap, d, 0.0, fa.FA_BF16, None)
+    assert st == fa.FA_ERR_INVALID
+    assert lib.fa_decode_noalloc(GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, 1, cap, d, 0.0, fa.FA_BF16,
+                                 None) == fa.FA_ERR_INVALID
+
+
+def test_decode_noalloc_within_its_array_reaches_the_runtime_without_a_gpu(lib):
+    # Sizes inside the array pass the size check and reach the CUDA runtime,
+    # which on a machine without a GPU fails the address lookup: FA_ERR_CUDA,
+    # not FA_ERR_INVALID.  Skipped where a GPU exists, since the fake pointers
+    # would then reach a kernel.
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers must not reach a GPU")
+    st = lib.fa_decode_noalloc(GOOD, GOOD, GOOD, GOOD, GOOD, None, 1016, 1, 8192, 128, 0.0,
+                               fa.FA_BF16, None)
+    assert st == fa.FA_ERR_CUDA

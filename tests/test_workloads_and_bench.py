@@ -111,3 +111,12 @@ def test_reference_arm_prints_one_json_line(workload, unit):
     assert d["config"]["workload"] == workload
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert np.isfinite(d["value"])
+
+
+def test_bench_line_names_the_workload_dtype():
+    import bench
+
+    W = workloads.WORKLOADS
+    assert bench.dtype_name(W["causal_prefill"].dtype) == "bf16"
+    assert bench.dtype_name(W["causal_prefill_fp16"].dtype) == "f16"
+    assert bench.dtype_name(W["single_head_fp32"].dtype) == "f32"

@@ -5,8 +5,11 @@ all device memory at start-up, plugin interfaces that pass only inputs and
 outputs), so this entry point keeps its scratch in an array built into the
 library.  Its results must match fa_decode's (the workspace version) on two
 calls in a row -- the second call reuses the array the first one filled.
-This file sorts last so that a run stopping at the first failure has already
-run every other test.
+A further test checks that calls after the first take no device memory.  Sizes
+beyond the array are refused on the host before any CUDA call; that check is
+tested without a GPU in test_abi_host.py, so no fake pointer ever reaches a GPU
+here.  This file sorts last so that a run stopping at the first failure has
+already run every other test.
 """
 import ctypes
 
@@ -52,13 +55,28 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
                                          d, 0.0, fa.FA_BF16, stream) == fa.FA_OK
 
 
-def test_noalloc_decode_rejects_sizes_beyond_its_array():
+def test_noalloc_decode_allocates_nothing_after_its_first_call():
+    # The point of the entry point: once the first call on a device has loaded
+    # the library's module (and with it the scratch array), further calls take
+    # no device memory.  The device's free bytes must not move across calls.
     import tiled_exact_attention_forward_b200 as fa
 
     lib = fa.library()
-    B, H, cap, d = 64, 32, 8192, 128   # needs ~17 MB of partials, more than the 8 MiB array
-    assert lib.fa_decode_workspace_size(B, H, cap, d) > 8 << 20
-    dummy = ctypes.c_void_p(0x100000)
-    st = lib.fa_decode_noalloc(dummy, dummy, dummy, dummy, dummy, None, B, H, cap, d, 0.0,
-                               fa.FA_BF16, None)
-    assert st == fa.FA_ERR_INVALID
+    B, H, cap, d = 4, 8, 2048, 128
+    q, kc, vc, lens = workloads.decode_inputs(B, H, cap, d, 1, cap, seed=23, device="cuda")
+    o = torch.empty_like(q)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def call():
+        assert lib.fa_decode_noalloc(_p(q), _p(kc), _p(vc), _p(lens), _p(o), None, B, H, cap, d,
+                                     0.0, fa.FA_BF16, stream) == fa.FA_OK
+
+    call()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert fa.device_status() == fa.FA_OK
+    assert free1 == free0, f"free device memory moved by {free0 - free1} bytes"

@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = (
     "fa_backward",
     "fa_get_device_status",
     "fa_selftest_wait_timeout",
+    "fa_selftest_exp2_poly",
     "fa_status_string",
     "fa_version",
 )
@@ -94,6 +95,8 @@ def _lib() -> ctypes.CDLL:
     lib.fa_backward.restype = I
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, P]
     lib.fa_selftest_wait_timeout.restype = I
+    lib.fa_selftest_exp2_poly.argtypes = [P, P, ctypes.c_longlong, P]
+    lib.fa_selftest_exp2_poly.restype = I
     lib.fa_get_device_status.argtypes = [P]
     lib.fa_get_device_status.restype = I
     lib.fa_status_string.argtypes = [I]

@@ -536,4 +536,6 @@ cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream) {
   return a.f16 ? launch_bwd_t<F16>(a, stream) : launch_bwd_t<Bf16>(a, stream);
 }
 
+cudaError_t take_status_bwd(unsigned int* out) { return take_local_status(out); }
+
 }  // namespace fa

@@ -13,8 +13,29 @@
 namespace fa {
 
 // Device status word (bit flags), read and cleared by fa_get_device_status().
+// The library is built as whole-program device code, one module per source
+// file (separate compilation would make ptxas ignore the per-warpgroup
+// register budgets of setmaxnreg), so each source file that launches kernels
+// has a status word of its own and exports a take_status_* accessor for it.
 enum : unsigned { kStatusTimeout = 1u };
-extern __device__ unsigned int g_status;
+namespace {
+__device__ unsigned int g_status = 0;
+
+// Read and clear this source file's status word.  Call after the work that may
+// have set it has completed.
+[[maybe_unused]] cudaError_t take_local_status(unsigned int* out) {
+  unsigned int word = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&word, g_status, sizeof(word));
+  if (e != cudaSuccess) return e;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *out = word;
+  return cudaSuccess;
+}
+}  // namespace
 
 // A wait that has not completed after this many SM clock cycles (about two
 // seconds at the B200's clocks) is treated as a hang: the kernel records
@@ -128,6 +149,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
       : "memory");
 }
 
+// Prefetch a 3-D tile of a tensor map into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 // 3-D tiled store shared -> global (bulk-group completion).
 __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int x, int y, int z) {
   asm volatile(
@@ -152,6 +181,19 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- register split
+// Move this warpgroup's per-thread register budget up or down (all four warps of
+// the warpgroup execute the same instruction).  The budgets of all warpgroups
+// must add up to at most the registers the block was launched with.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------- tcgen05 / TMEM

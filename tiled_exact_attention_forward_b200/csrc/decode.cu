@@ -230,4 +230,6 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t take_status_decode(unsigned int* out) { return take_local_status(out); }
+
 }  // namespace fa

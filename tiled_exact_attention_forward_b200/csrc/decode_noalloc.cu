@@ -10,16 +10,20 @@
 // keeps the partials in a fixed array compiled into the library instead, so a
 // call allocates nothing.
 //
-// The array lives in device global memory on every GPU that loads the
-// library, for the life of the process.  Its host-side name is only a shadow
-// of the device array, so the device address is looked up with
-// cudaGetSymbolAddress -- once per device, on the first call made while that
-// device is current.  That first call should come before any stream capture.
+// The array lives in device global memory.  With lazy module loading (the
+// CUDA 12 default) it is reserved on a device by the first call made there
+// (or at library load when CUDA_MODULE_LOADING=EAGER) and held until the
+// process exits.  Its host-side name is only a shadow of the device array, so
+// every call asks the runtime for the device address in the CURRENT context
+// with cudaGetSymbolAddress.  The address belongs to a context, not to a
+// device: after cudaDeviceReset, or with another context made current on the
+// same device, the module is loaded again at a new address, which is why no
+// address is kept between calls.  Once the module is loaded the lookup is a
+// table search that does not synchronise.  The first call on each device
+// loads the module: make it at start-up, before any stream capture.
 // All calls share the array: two calls whose kernels overlap on the GPU race
 // on it.  Nothing in it needs clearing between calls, because every partial
 // the combine step reads is written earlier in the same call.
-#include <mutex>
-
 #include "../../include/fa.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -27,27 +31,6 @@
 namespace {
 
 static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[FA_DECODE_NOALLOC_SCRATCH_BYTES];
-
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device.
-cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return cudaSuccess;
-}
 
 }  // namespace
 
@@ -57,6 +40,7 @@ extern "C" fa_status fa_decode_noalloc(const void* q, const void* kcache, const 
   const size_t need = fa_decode_workspace_size(B, H, cap, d);
   if (need == 0 || need > static_cast<size_t>(FA_DECODE_NOALLOC_SCRATCH_BYTES)) return FA_ERR_INVALID;
   void* scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaGetSymbolAddress(&scratch, g_decode_noalloc_scratch) != cudaSuccess || scratch == nullptr)
+    return FA_ERR_CUDA;
   return fa_decode(q, kcache, vcache, seqlens, o, lse, B, H, cap, d, scale, dtype, scratch, need, stream);
 }

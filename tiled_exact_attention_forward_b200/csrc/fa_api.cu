@@ -32,7 +32,7 @@ bool sizes_ok(long long B, long long H, long long N) {
 
 extern "C" {
 
-int fa_version(void) { return 102; }
+int fa_version(void) { return 103; }
 
 const char* fa_status_string(fa_status s) {
   switch (s) {
@@ -212,20 +212,26 @@ fa_status fa_selftest_wait_timeout(long long limit_cycles, void* stream) {
   return from_cuda(fa::launch_selftest_wait_timeout(limit_cycles, static_cast<cudaStream_t>(stream)));
 }
 
+fa_status fa_selftest_exp2_poly(const float* x, float* y, long long n, void* stream) {
+  if (!x || !y || n < 1 || !aligned(x, 4) || !aligned(y, 4)) return FA_ERR_INVALID;
+  return from_cuda(fa::launch_selftest_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 fa_status fa_get_device_status(void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return FA_ERR_CUDA;
+  // Each source file's kernels record into a status word of their own; gather
+  // (and clear) all of them.
   unsigned int word = 0;
-  e = cudaMemcpyFromSymbol(&word, fa::g_status, sizeof(word));
-  if (e != cudaSuccess) return FA_ERR_CUDA;
-  if (word != 0) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(zero));
+  for (auto take : {fa::take_status_host, fa::take_status_fwd_tc, fa::take_status_bwd, fa::take_status_decode}) {
+    unsigned int w = 0;
+    e = take(&w);
     if (e != cudaSuccess) return FA_ERR_CUDA;
-    if (word & fa::kStatusTimeout) return FA_ERR_TIMEOUT;
-    if (word & fa::kStatusBadBlock) return FA_ERR_INVALID;
+    word |= w;
   }
+  if (word & fa::kStatusTimeout) return FA_ERR_TIMEOUT;
+  if (word & fa::kStatusBadBlock) return FA_ERR_INVALID;
   return FA_OK;
 }
 

@@ -11,7 +11,7 @@
 
 namespace fa {
 
-__device__ unsigned int g_status = 0;
+cudaError_t take_status_host(unsigned int* out) { return take_local_status(out); }
 
 namespace {
 
@@ -122,7 +122,29 @@ __global__ void selftest_wait_timeout_kernel(long long limit_cycles) {
   (void)ok;
 }
 
+// Evaluates the forward's exp2 cubic (exp2_poly_pair) on an array, two values
+// per thread exactly as the softmax feeds it, so a test can hold the device
+// function to its stated error bound.
+__global__ void selftest_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long stride = 2LL * gridDim.x * blockDim.x;
+  for (long long i = 2LL * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x); i < n; i += stride) {
+    const bool two = i + 1 < n;
+    const uint64_t r = exp2_poly_pair(f2_pack(x[i], two ? x[i + 1] : 0.f));
+    float r0, r1;
+    f2_unpack(r, r0, r1);
+    y[i] = r0;
+    if (two) y[i + 1] = r1;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream) {
+  const long long pairs = (n + 1) / 2;
+  const long long blocks = (pairs + 255) / 256;
+  selftest_exp2_poly_kernel<<<static_cast<unsigned>(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, cudaStream_t stream) {
   selftest_wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_cycles);

@@ -662,4 +662,6 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+cudaError_t take_status_fwd_tc(unsigned int* out) { return take_local_status(out); }
+
 }  // namespace fa

@@ -94,11 +94,18 @@ cudaError_t set_max_dynamic_smem(const void* func, size_t bytes);
 // Number of SMs of the current device (cached per device).
 cudaError_t sm_count(int* out);
 
+// Read and clear the device status word of each source file that has one.
+cudaError_t take_status_host(unsigned int* out);
+cudaError_t take_status_fwd_tc(unsigned int* out);
+cudaError_t take_status_bwd(unsigned int* out);
+cudaError_t take_status_decode(unsigned int* out);
+
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
 cudaError_t launch_selftest_wait_timeout(long long limit_cycles, cudaStream_t stream);
+cudaError_t launch_selftest_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 
 }  // namespace fa
