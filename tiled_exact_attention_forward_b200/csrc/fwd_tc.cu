@@ -17,20 +17,32 @@
 //     or window mask hides from every row of a query tile are never loaded
 //     for it; only tiles that straddle a mask edge (or the ragged end of the
 //     sequence) get the per-element mask.
-//   * Warp roles (608 threads): warps 0-7 and 8-15 are the softmax warps of
-//     query tiles 0 and 1 (two threads per query row = TMEM lane, one per
-//     64-column half, in warps i and i + 4 of the tile, exchanging row max and
-//     sum through shared memory behind a 64-thread barrier per warp pair);
-//     warp 16 allocates tensor memory and issues every MMA from one thread;
-//     warp 17 streams K/V through the ring by TMA and warp 18 loads the Q
-//     tiles, each as soon as its slot frees.
+//   * Warp roles (512 threads, four warpgroups):
+//       warpgroups 0 and 1 -- the softmax of query tiles 0 and 1: one thread
+//         per query row (= TMEM lane), all 128 score columns in registers, so
+//         the row max and sum need no exchange between threads;
+//       warpgroup 2 -- the epilogue: reads O out of TMEM, divides by the row
+//         sum, stores O (16-bit) and lse, so the softmax warps go straight on
+//         to the next item's first tile;
+//       warpgroup 3 -- warp 12 allocates tensor memory and issues every MMA,
+//         warp 13 streams K/V through the ring by TMA, warp 14 loads the Q
+//         tiles (each as soon as its slot frees) and prefetches the next item's
+//         Q tiles into L2.
+//     The MMA warp runs its whole loop warp-uniformly and issues each MMA and
+//     commit from one elected lane; a single thread issues tcgen05.mma barely
+//     faster than the tensor core retires a 128x128x16 step (measured), and a
+//     warp that branches with one active lane issues slower still, so the
+//     issuer keeps its control flow uniform and its waits and commits few:
+//     per key tile one wait per K/V ring entry (TMA data: no tcgen05 fence),
+//     one P wait per tile, one commit per S and per ring entry.
+//     Registers are split with setmaxnreg: 192 per softmax thread, 64 per
+//     epilogue thread and 64 for warpgroup 3 (256*192 + 128*64 + 128*64 =
+//     65536, the block's launch budget of 512 threads x 128).  The host
+//     refuses to launch unless the compiled kernel has exactly that budget.
 //   * Items are dealt to a persistent grid of one CTA per SM, heaviest first.
 //     With a causal mask tile 0 of an item ends one key tile before tile 1;
 //     S_0 of the next item's first key tile is then issued at once, so tile
-//     0's softmax warps do not idle across the item boundary.  (Issuing the
-//     two tiles' MMAs independently -- polled, or from two threads -- was
-//     measured slower: the two softmaxes then overlap and contend for the
-//     same pipes, where the fixed order below keeps them alternating.)
+//     0's softmax warps do not idle across the item boundary.
 //   * Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.
 //     The softmax writes P (16-bit pairs) over the first 64 columns of its S
 //     tile, and O += P V reads P straight from tensor memory (A operand in
@@ -44,10 +56,9 @@
 //     when the new row max exceeds it by more than 2^8 in exp2 units; P is
 //     then at most 256, exact in the final O / l.
 //   * exp2 with scale*log2(e) folded into one packed (f32x2) FMA per score
-//     pair.  One pair in eight takes 2^x from a cubic on the FMA pipe instead
-//     of the special-function unit, whose rate (16 results per clock per SM)
-//     otherwise equals the MMA rate for d = 128; more than that loads the FMA
-//     and issue slots more than it relieves the ex2 unit (measured).
+//     pair.  A share of the pairs takes 2^x from a cubic on the FMA pipe
+//     instead of the special-function unit, whose rate (16 results per clock
+//     per SM) otherwise equals the MMA rate for d = 128.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -61,13 +72,24 @@ constexpr int D = 128;                  // head dimension
 constexpr int NS = 4;                   // K/V ring stages (K and V tiles interleaved)
 constexpr int TILE_BYTES = BM * D * 2;  // one 128 x 128 16-bit tile = 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;  // one 64-column half (a 128-byte-swizzled box)
-constexpr int NUM_THREADS = 608;     // 16 softmax warps + MMA warp + K/V TMA warp + Q TMA warp
-constexpr int WG_THREADS = 256;      // one softmax warpgroup pair per query tile
-constexpr int MMA_WARP = 16;
-constexpr int TMA_WARP = 17;         // K/V stream
-constexpr int QLD_WARP = 18;         // Q tiles: loaded as soon as their slot frees
+constexpr int NUM_THREADS = 512;     // 4 warpgroups: softmax 0, softmax 1, epilogue, MMA/TMA
+constexpr int WG_THREADS = 128;      // one warpgroup: one thread per row of a query tile
+constexpr int EPI_WG = 2;            // epilogue warpgroup (warps 8-11)
+constexpr int MMA_WARP = 12;
+constexpr int TMA_WARP = 13;         // K/V stream
+constexpr int QLD_WARP = 14;         // Q tiles: loaded as soon as their slot frees
+constexpr int kSoftmaxRegs = 192;    // 128 scores + exp2 pipeline, no spills
+constexpr int kEpilogueRegs = 64;
+constexpr int kOtherRegs = 64;
+constexpr int kLaunchRegs = 128;     // 65536 / NUM_THREADS: what the split draws on
+static_assert(2 * WG_THREADS * kSoftmaxRegs + WG_THREADS * kEpilogueRegs + WG_THREADS * kOtherRegs <=
+                  NUM_THREADS * kLaunchRegs,
+              "register split exceeds the launch budget");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPolyPairs = 1;  // of every 8 score pairs, those exponentiated on the FMA pipe
+#ifndef FA_FWD_POLY_PAIRS
+#define FA_FWD_POLY_PAIRS 1
+#endif
+constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;  // of every 8 score pairs, those exponentiated on the FMA pipe
 
 struct Smem {
   // 1024-byte aligned by construction (the dynamic buffer is aligned at runtime).
@@ -78,14 +100,15 @@ struct Smem {
   uint64_t kv_full[NS];
   uint64_t kv_empty[NS];
   uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_full[2];
-  uint64_t o_free[2];
+  uint64_t p_full[2];   // P stored in TMEM (and O rescaled if it had to be)
+  uint64_t o_full[2];   // last PV of an item complete
+  uint64_t o_free[2];   // epilogue has read O out of TMEM
+  uint64_t st_full[2];  // softmax has published the item's row statistics
+  uint64_t st_empty[2]; // epilogue has read them
   uint64_t mma_done;
-  // Row statistics exchanged between the two threads of a row (column halves):
-  // [tile][step parity][half][row].
-  float xmax[2][2][2][BM];
-  float xsum[2][2][BM];
+  // Row statistics of a finished item, softmax -> epilogue: [tile][row].
+  float stat_m[2][BM];
+  float stat_l[2][BM];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -138,32 +161,66 @@ __device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
-// S = Q K^T: Q and K tiles K-major ([64-column half][128 rows][64 cols]); a K step
-// of 16 columns is 32 bytes inside a half, the second half 16 KiB further on.
-template <class T>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo) {
-  constexpr uint32_t idesc = idesc_f32acc<T>(BM, BN, 0, 0);
-  constexpr uint32_t hi = desc_hi(1024);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
-    mma_ss(d_tmem, desc_of(q_lo + off, hi), desc_of(k_lo + off, hi), idesc, kk > 0 ? 1u : 0u);
-  }
+// One kind::f16 MMA with both operands in shared memory; the descriptors are
+// the bases plus compile-time offsets (in 16-byte units) added inside the asm,
+// so an unrolled chain costs a few instructions per MMA and no registers for
+// precomputed descriptors.  The whole warp executes it and one elected lane
+// issues the MMA: the issuing warp's control flow stays uniform (a warp that
+// runs its loop on one lane issues MMAs measurably slower).
+template <uint32_t OFF_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
+__device__ __forceinline__ void mma_ss_at(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t acc_in) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
+      "add.s64 ad, %1, %4;\n\t"
+      "add.s64 bd, %2, %5;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %6, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(OFF_A), "n"(OFF_B), "n"(IDESC)
+      : "memory");
+}
+// The same with A read from tensor memory at a compile-time column offset.
+template <uint32_t COL_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
+__device__ __forceinline__ void mma_ts_at(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t acc_in) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 at;\n\t.reg .b64 bd;\n\t"
+      "add.u32 at, %1, %4;\n\t"
+      "add.s64 bd, %2, %5;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %6, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(COL_A), "n"(OFF_B), "n"(IDESC)
+      : "memory");
 }
 
-// O += P V: V tile MN-major ([64-column half][128 keys][64 cols]); a K step of 16
-// keys is 16 rows = 2 KiB.  P of keys [64h, 64h + 64) sits in S columns
-// [64h, 64h + 32) (16-bit pairs).
-template <class T>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo, bool accumulate) {
+// tcgen05.commit from one elected lane of a warp that executes it uniformly.
+__device__ __forceinline__ void commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
+// S = Q K^T: Q and K tiles K-major ([64-column half][128 rows][64 cols]); a K step
+// of 16 columns is 32 bytes inside a half, the second half 16 KiB further on.
+template <class T, int KK = 0>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+  constexpr uint32_t off = ((KK >> 2) * HALF_BYTES + (KK & 3) * 32) >> 4, acc = KK > 0 ? 1u : 0u;
+  constexpr uint32_t idesc = idesc_f32acc<T>(BM, BN, 0, 0);
+  mma_ss_at<off, off, idesc, acc>(d_tmem, q_desc, k_desc, 0u);
+  if constexpr (KK + 1 < D / 16) issue_qk<T, KK + 1>(d_tmem, q_desc, k_desc);
+}
+
+// O += P V: V tile MN-major ([64-column half][128 keys][64 cols]); a K step of
+// 16 keys is 16 rows = 2 KiB.  P of keys [2c, 2c + 1] sits in S column c (16-bit
+// pairs), so the A operand of K step kk starts at column 8 kk.  The first step
+// accumulates only when `accumulate` is set (the first PV of an item overwrites O).
+template <class T, int KK = 0>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, uint32_t accumulate) {
+  constexpr uint32_t col = KK * 8, off = (KK * 16 * 128) >> 4, acc = KK > 0 ? 1u : 0u;
   constexpr uint32_t idesc = idesc_f32acc<T>(BM, D, 0, 1);
-  constexpr uint32_t hi = desc_hi(1024);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint32_t a_col = (kk >> 2) * 64 + (kk & 3) * 8;
-    mma_ts(d_tmem, p_tmem + a_col, desc_of(v_lo + ((kk * 16 * 128) >> 4), hi), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
-  }
+  mma_ts_at<col, off, idesc, acc>(d_tmem, p_tmem, v_desc, accumulate);
+  if constexpr (KK + 1 < BN / 16) issue_pv<T, KK + 1>(d_tmem, p_tmem, v_desc, accumulate);
 }
 
 // One unit of work: two 128-row query tiles (rows [256p, 256p + 256)) of one
@@ -232,6 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int wg = warp >> 2;
   const int BH = args.B * args.H;
   const int n = args.N;
   const int num_pairs = (n + 2 * BM - 1) / (2 * BM);
@@ -248,6 +306,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&sm.p_full[t]), WG_THREADS);
       mbar_init(smem_u32(&sm.o_full[t]), 1);
       mbar_init(smem_u32(&sm.o_free[t]), WG_THREADS);
+      mbar_init(smem_u32(&sm.st_full[t]), WG_THREADS);
+      mbar_init(smem_u32(&sm.st_empty[t]), WG_THREADS);
     }
     for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&sm.kv_full[s]), 1);
@@ -272,257 +332,312 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == QLD_WARP) {
-    // ------------------------------------------------------------ Q loader
-    // A warp of its own, so the next item's Q tile goes out as soon as the last
-    // S MMA of the current item has read the slot, ahead of the K/V stream.
-    if (lane == 0) {
-      int nq[2] = {0, 0};  // Q tiles loaded so far, per slot
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int lin = item_of(k, total);
-        if (lin < 0) break;
-        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!active(it, t)) continue;
-          if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
-          if (!ok) break;
-          const uint32_t bar = smem_u32(&sm.q_full[t]);
-          mbar_arrive_expect_tx(bar, TILE_BYTES);
-          tma_load_3d(smem_u32(sm.q[t]), &tm_q, bar, 0, it.r0[t], it.bh);
-          tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, it.r0[t], it.bh);
-          ++nq[t];
-        }
-      }
-      for (int t = 0; t < 2; ++t)
-        if (nq[t] > 0) mbar_wait_drain(smem_u32(&sm.q_full[t]), (nq[t] - 1) & 1);
-    }
-  } else if (warp == TMA_WARP) {
-    // ------------------------------------------------------------ K/V producer
-    if (lane == 0) {
-      int kvi = 0;         // K/V ring fills so far (K and V interleaved)
-      bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int lin = item_of(k, total);
-        if (lin < 0) break;
-        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
-        for (int idx = 0; ok && idx < 2 * (it.hi - it.lo); ++idx, ++kvi) {
-          const int s = kvi % NS;
-          if (kvi >= NS) ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((kvi / NS) - 1) & 1, abort_flag);
-          if (!ok) break;
-          const int j = it.lo + (idx >> 1);
-          const CUtensorMap* tm = (idx & 1) ? &tm_v : &tm_k;
-          const uint32_t bar = smem_u32(&sm.kv_full[s]);
-          mbar_arrive_expect_tx(bar, TILE_BYTES);
-          tma_load_3d(smem_u32(sm.kv[s]), tm, bar, 0, j * BN, it.bh);
-          tma_load_3d(smem_u32(sm.kv[s]) + HALF_BYTES, tm, bar, 64, j * BN, it.bh);
-        }
-      }
-      // Drain: every copy issued must land before the CTA may exit.
-      for (int i = max(0, kvi - NS); i < kvi; ++i) mbar_wait_drain(smem_u32(&sm.kv_full[i % NS]), (i / NS) & 1);
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t tS[2] = {tmem + 0, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 384};
-      // Descriptor low words of the Q slots (K-major, leading-byte offset 16).
-      const uint32_t q_s[2] = {desc_lo(smem_u32(sm.q[0]), 16), desc_lo(smem_u32(sm.q[1]), 16)};
-      int nq[2] = {0, 0};    // Q tiles consumed, per slot
-      bool q_ready[2] = {false, false};  // slot t holds the tile now in use and was waited for
-      int npv[2] = {0, 0};   // PV MMAs issued, per tile slot (p_full phase)
-      int nout[2] = {0, 0};  // items finished, per tile slot (o_full / o_free phase)
-      int kvi = 0;
-      bool ok = true;
-      bool s0_ahead = false;  // S_0(lo) of this item was issued during the previous item
-      auto stage_of = [&](int i) { return i % NS; };
-      auto parity_of = [&](int i) { return static_cast<uint32_t>((i / NS) & 1); };
-      // S_t(j) of item `it`: waits for the item's Q tile on first use; the item's last
-      // S_t releases the Q slot to the loader.
-      auto issue_s = [&](const Item& it, int t, int j, uint32_t ks) -> bool {
-        if (!q_ready[t]) {
-          if (!mbar_wait(smem_u32(&sm.q_full[t]), nq[t] & 1, abort_flag)) return false;
-          ++nq[t];
-          q_ready[t] = true;
-          tc_fence_after();
-        }
-        issue_qk<T>(tS[t], q_s[t], ks);
-        tc_commit(smem_u32(&sm.s_full[t]));
-        if (j == it.hi_t[t] - 1) {
-          tc_commit(smem_u32(&sm.q_empty[t]));
-          q_ready[t] = false;
-        }
-        return true;
-      };
-      for (int k = 0; ok; ++k) {
-        const int lin = item_of(k, total);
-        if (lin < 0) break;
-        const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
-        auto act = [&](int t, int j) { return j >= it.lo_t[t] && j < it.hi_t[t]; };
-        // PV_t(j): the first one of an item overwrites O_t, so the previous item's
-        // epilogue must have read it out; the last one publishes O_t.
-        auto issue_o = [&](int t, int j, uint32_t vs) -> bool {
-          if (j == it.lo_t[t] && nout[t] > 0) {
-            if (!mbar_wait(smem_u32(&sm.o_free[t]), (nout[t] - 1) & 1, abort_flag)) return false;
+  if (wg == 3) {
+    regs_dec<kOtherRegs>();
+    if (warp == QLD_WARP) {
+      // ---------------------------------------------------------- Q loader
+      // A warp of its own, so the next item's Q tile goes out as soon as the last
+      // S MMA of the current item has read the slot, ahead of the K/V stream.  The
+      // item after that has its Q tiles prefetched into L2 meanwhile.
+      if (lane == 0) {
+        int nq[2] = {0, 0};  // Q tiles loaded so far, per slot
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int lin = item_of(k, total);
+          if (lin < 0) break;
+          const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
+          const int lin2 = item_of(k + 1, total);
+          if (lin2 >= 0) {
+            const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
+            for (int t = 0; t < 2; ++t) {
+              if (!active(nx, t)) continue;
+              tma_prefetch_l2_3d(&tm_q, 0, nx.r0[t], nx.bh);
+              tma_prefetch_l2_3d(&tm_q, 64, nx.r0[t], nx.bh);
+            }
           }
-          if (!mbar_wait(smem_u32(&sm.p_full[t]), npv[t] & 1, abort_flag)) return false;
-          tc_fence_after();
-          issue_pv<T>(tO[t], tS[t], vs, j > it.lo_t[t]);
-          ++npv[t];
-          if (j == it.hi_t[t] - 1) {
-            tc_commit(smem_u32(&sm.o_full[t]));
-            ++nout[t];
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (!active(it, t)) continue;
+            if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
+            if (!ok) break;
+            const uint32_t bar = smem_u32(&sm.q_full[t]);
+            mbar_arrive_expect_tx(bar, TILE_BYTES);
+            tma_load_3d(smem_u32(sm.q[t]), &tm_q, bar, 0, it.r0[t], it.bh);
+            tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, it.r0[t], it.bh);
+            ++nq[t];
+          }
+        }
+        for (int t = 0; t < 2; ++t)
+          if (nq[t] > 0) mbar_wait_drain(smem_u32(&sm.q_full[t]), (nq[t] - 1) & 1);
+      }
+    } else if (warp == TMA_WARP) {
+      // ---------------------------------------------------------- K/V producer
+      if (lane == 0) {
+        int kvi = 0;  // K/V ring fills so far (K and V interleaved)
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+          const int lin = item_of(k, total);
+          if (lin < 0) break;
+          const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
+          for (int idx = 0; ok && idx < 2 * (it.hi - it.lo); ++idx, ++kvi) {
+            const int s = kvi % NS;
+            if (kvi >= NS) ok = mbar_wait(smem_u32(&sm.kv_empty[s]), ((kvi / NS) - 1) & 1, abort_flag);
+            if (!ok) break;
+            const int j = it.lo + (idx >> 1);
+            const CUtensorMap* tm = (idx & 1) ? &tm_v : &tm_k;
+            const uint32_t bar = smem_u32(&sm.kv_full[s]);
+            mbar_arrive_expect_tx(bar, TILE_BYTES);
+            tma_load_3d(smem_u32(sm.kv[s]), tm, bar, 0, j * BN, it.bh);
+            tma_load_3d(smem_u32(sm.kv[s]) + HALF_BYTES, tm, bar, 64, j * BN, it.bh);
+          }
+        }
+        // Drain: every copy issued must land before the CTA may exit.
+        for (int i = max(0, kvi - NS); i < kvi; ++i) mbar_wait_drain(smem_u32(&sm.kv_full[i % NS]), (i / NS) & 1);
+      }
+    } else if (warp == MMA_WARP) {
+      // ---------------------------------------------------------- MMA issuer
+      // The whole warp runs this loop (warp-uniform waits); MMAs and commits are
+      // issued by one elected lane.
+      {
+        // Phase bits of the per-tile barriers, bit t for tile slot t:
+        //   Q_PH  q_full phase to wait for next      QRDY  slot t holds the tile in use
+        //   PV_PH p_full phase                       O_USED an item has used O_t before
+        //   O_PH  o_free phase of the last item that finished on tile t
+        enum : uint32_t { Q_PH = 0, QRDY = 2, PV_PH = 4, O_USED = 6, O_PH = 8 };
+        uint32_t ph = 0;
+        int kvi = 0;
+        bool ok = true;
+        bool s0_ahead = false;  // S_0(lo) of this item was issued during the previous item
+        auto bit = [&](uint32_t b) { return (ph >> b) & 1u; };
+        auto stage_addr = [&](int i) { return smem_u32(sm.kv[i % NS]); };
+        // K/V tiles arrive by TMA: the barrier's completion orders the copy before
+        // the MMAs' reads (no tcgen05 fence needed, unlike data another thread's
+        // tcgen05 instructions produced).
+        auto wait_kv = [&](int i) {
+          return mbar_wait_warp(smem_u32(&sm.kv_full[i % NS]), static_cast<uint32_t>((i / NS) & 1), abort_flag);
+        };
+        // S_t(j): waits for the item's Q tile on first use; the item's last S_t
+        // (last == true) releases the Q slot to the loader.
+        auto issue_s = [&](int t, bool last, uint32_t k_addr) -> bool {
+          if (!bit(QRDY + t)) {
+            if (!mbar_wait_warp(smem_u32(&sm.q_full[t]), bit(Q_PH + t), abort_flag)) return false;
+            ph ^= 1u << (Q_PH + t);
+            ph |= 1u << (QRDY + t);
+          }
+          issue_qk<T>(tmem + 128 * t, desc_of(desc_lo(smem_u32(sm.q[t]), 16), desc_hi(1024)),
+                      desc_of(desc_lo(k_addr, 16), desc_hi(1024)));
+          commit_elect(smem_u32(&sm.s_full[t]));
+          if (last) {
+            commit_elect(smem_u32(&sm.q_empty[t]));
+            ph &= ~(1u << (QRDY + t));
           }
           return true;
         };
-        if (it.hi <= it.lo) {  // no active tile: nothing to issue
-          if (OFFSET) continue;
-          break;
-        }
-        // Prologue: S_t(lo) for both tiles (S_0(lo) may already be in flight).
-        ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi)]), parity_of(kvi), abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        {
-          const uint32_t ks = desc_lo(smem_u32(sm.kv[stage_of(kvi)]), 16);
-          for (int t = 0; t < 2 && ok; ++t)
-            if (act(t, it.lo) && !(t == 0 && s0_ahead)) ok = issue_s(it, t, it.lo, ks);
-          if (!ok) break;
-          tc_commit(smem_u32(&sm.kv_empty[stage_of(kvi)]));
+        // PV_t(j) once P_t(j) is in TMEM.  The first PV of an item (first == true)
+        // overwrites O_t, so the epilogue must have read the previous item's O_t
+        // out; the last one (last == true) publishes O_t.
+        auto issue_o = [&](int t, bool first, bool last, uint32_t v_addr) -> bool {
+          if (first && bit(O_USED + t)) {
+            if (!mbar_wait_warp(smem_u32(&sm.o_free[t]), bit(O_PH + t), abort_flag)) return false;
+            ph ^= 1u << (O_PH + t);
+          }
+          const uint64_t vs = desc_of(desc_lo(v_addr, HALF_BYTES), desc_hi(1024));
+          if (!mbar_wait_warp(smem_u32(&sm.p_full[t]), bit(PV_PH + t), abort_flag)) return false;
+          tc_fence_after();
+          issue_pv<T>(tmem + 256 + 128 * t, tmem + 128 * t, vs, first ? 0u : 1u);
+          ph ^= 1u << (PV_PH + t);
+          if (last) {
+            commit_elect(smem_u32(&sm.o_full[t]));
+            ph |= 1u << (O_USED + t);
+          }
+          return true;
+        };
+        for (int k = 0; ok; ++k) {
+          const int lin = item_of(k, total);
+          if (lin < 0) break;
+          const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
+          auto act = [&](int t, int j) { return j >= it.lo_t[t] && j < it.hi_t[t]; };
+          if (it.hi <= it.lo) {  // no active tile: nothing to issue
+            if (OFFSET) continue;
+            break;
+          }
+          // Prologue: S_t(lo) for both tiles (S_0(lo) may already be in flight).
+          if (!(ok = wait_kv(kvi))) break;
+          if (act(0, it.lo) && !s0_ahead && !(ok = issue_s(0, it.lo == it.hi_t[0] - 1, stage_addr(kvi)))) break;
+          if (act(1, it.lo) && !(ok = issue_s(1, it.lo == it.hi_t[1] - 1, stage_addr(kvi)))) break;
+          commit_elect(smem_u32(&sm.kv_empty[kvi % NS]));
           ++kvi;
           s0_ahead = false;
-        }
-        for (int j = it.lo; ok && j < it.hi; ++j) {
-          const int vidx = kvi;            // V_j
-          const int nidx = kvi + 1;        // K_{j+1}
-          const bool has_next = j + 1 < it.hi;
-          ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(vidx)]), parity_of(vidx), abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vs = desc_lo(smem_u32(sm.kv[stage_of(vidx)]), HALF_BYTES);
-          if (act(0, j) && !(ok = issue_o(0, j, vs))) break;
-          uint32_t ks = 0;
-          if (has_next) {
-            ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(nidx)]), parity_of(nidx), abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            ks = desc_lo(smem_u32(sm.kv[stage_of(nidx)]), 16);
-            if (act(0, j + 1) && !(ok = issue_s(it, 0, j + 1, ks))) break;
-          }
-          if (act(1, j) && !(ok = issue_o(1, j, vs))) break;
-          tc_commit(smem_u32(&sm.kv_empty[stage_of(vidx)]));
-          if (has_next) {
-            if (act(1, j + 1) && !(ok = issue_s(it, 1, j + 1, ks))) break;
-            tc_commit(smem_u32(&sm.kv_empty[stage_of(nidx)]));
-          }
-          kvi += has_next ? 2 : 1;
-          // Causal masks end tile 0 one key tile before tile 1.  Its softmax warps
-          // would then idle until tile 1 finishes, so S_0 of the next item's first
-          // key tile goes out now: K(lo') is the ring entry after V(hi - 1), and
-          // ring entry kvi + 1 - NS has been consumed already.
-          if (j == it.hi - 2 && it.has1 && !act(0, j + 1)) {
-            const int lin2 = item_of(k + 1, total);
-            if (lin2 >= 0) {
-              const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
-              if (active(nx, 0) && nx.lo_t[0] == nx.lo) {
-                ok = mbar_wait(smem_u32(&sm.kv_full[stage_of(kvi + 1)]), parity_of(kvi + 1), abort_flag);
-                if (!ok) break;
-                tc_fence_after();
-                if (!(ok = issue_s(nx, 0, nx.lo, desc_lo(smem_u32(sm.kv[stage_of(kvi + 1)]), 16)))) break;
-                s0_ahead = true;
+          for (int j = it.lo; ok && j < it.hi; ++j) {
+            const int vidx = kvi;      // V_j
+            const int nidx = kvi + 1;  // K_{j+1}
+            const bool has_next = j + 1 < it.hi;
+            if (!(ok = wait_kv(vidx))) break;
+            if (act(0, j) && !(ok = issue_o(0, j == it.lo_t[0], j == it.hi_t[0] - 1, stage_addr(vidx)))) break;
+            if (has_next) {
+              if (!(ok = wait_kv(nidx))) break;
+              if (act(0, j + 1) && !(ok = issue_s(0, j + 1 == it.hi_t[0] - 1, stage_addr(nidx)))) break;
+            }
+            if (act(1, j) && !(ok = issue_o(1, j == it.lo_t[1], j == it.hi_t[1] - 1, stage_addr(vidx)))) break;
+            commit_elect(smem_u32(&sm.kv_empty[vidx % NS]));
+            if (has_next) {
+              if (act(1, j + 1) && !(ok = issue_s(1, j + 1 == it.hi_t[1] - 1, stage_addr(nidx)))) break;
+              commit_elect(smem_u32(&sm.kv_empty[nidx % NS]));
+            }
+            kvi += has_next ? 2 : 1;
+            // Causal masks end tile 0 one key tile before tile 1.  Its softmax warps
+            // would then idle until tile 1 finishes, so S_0 of the next item's first
+            // key tile goes out now: K(lo') is the ring entry after V(hi - 1), and
+            // ring entry kvi + 1 - NS has been consumed already.
+            if (j == it.hi - 2 && it.has1 && !act(0, j + 1)) {
+              const int lin2 = item_of(k + 1, total);
+              if (lin2 >= 0) {
+                const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
+                if (active(nx, 0) && nx.lo_t[0] == nx.lo) {
+                  const bool last = nx.lo == nx.hi_t[0] - 1;
+                  if (!(ok = wait_kv(kvi + 1))) break;
+                  if (!(ok = issue_s(0, last, stage_addr(kvi + 1)))) break;
+                  s0_ahead = true;
+                }
               }
             }
           }
         }
+        // All MMAs issued by this warp must complete before TMEM is freed.
+        commit_elect(smem_u32(&sm.mma_done));
+        mbar_wait_drain(smem_u32(&sm.mma_done), 0);
       }
-      // All MMAs issued by this thread must complete before TMEM is freed.
-      tc_commit(smem_u32(&sm.mma_done));
-      mbar_wait_drain(smem_u32(&sm.mma_done), 0);
+      __syncwarp();
     }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ softmax warps
-    // 8 warps per query tile: warp i of the tile reads TMEM lanes 32*(i%4).. (one row
-    // per thread) and columns [64h, 64h + 64) with h = i/4, so two threads share a
-    // row and exchange its max and sum through shared memory.
-    const int t = warp >> 3;         // query tile slot
-    const int wi = warp & 7;
-    const int hc = wi >> 2;          // column half
-    const int row = (wi & 3) * 32 + lane;
-    // The two threads of a row sit in warps wi and wi + 4 (same TMEM lanes); only
-    // that warp pair exchanges, on a 64-thread named barrier of its own.
-    const int bar_id = 3 + 4 * t + (wi & 3);
-    constexpr int kBarThreads = 64;
-    const uint32_t lane_off = static_cast<uint32_t>((wi & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128 + 64 * hc;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128 + 64 * hc;
-    const float sl2 = args.scale_log2;
-    int ns = 0;    // S tiles consumed (s_full phase)
-    int nout = 0;  // items finished (o_full phase)
+  } else if (wg == EPI_WG) {
+    // ------------------------------------------------------------ epilogue
+    // Thread = one row of each query tile (TMEM lane 32 (warp % 4) + lane): waits
+    // for the item's last PV and the softmax's row statistics, reads O_t out of
+    // TMEM in 32-column chunks, frees O_t for the next item, and stores O / l in
+    // 16 bits and lse = m * scale + ln l.
+    regs_dec<kEpilogueRegs>();
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int nfull[2] = {0, 0};
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int lin = item_of(k, total);
       if (lin < 0) break;
       const Item item = make_item<OFFSET>(lin, BH, num_pairs, geo);
-      if (t == 1 && !item.has1) continue;
-      const int r0 = item.r0[t];
-      const int row_g = r0 + row;
-      if (OFFSET && !item.active(t)) {
-        // No row of this tile sees a key: O = 0, lse = -inf.
-        if (row_g < n) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.o) +
-                                                (static_cast<size_t>(item.bh) * n + row_g) * D + 64 * hc);
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (t == 1 && !item.has1) continue;
+        const int row_g = item.r0[t] + row;
+        uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) + (static_cast<size_t>(item.bh) * n + row_g) * D;
+        if (OFFSET && !item.active(t)) {
+          // No row of this tile sees a key: O = 0, lse = -inf.
+          if (row_g < n) {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
 #pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
-          if (hc == 0 && args.lse != nullptr) args.lse[static_cast<size_t>(item.bh) * n + row_g] = -INFINITY;
+            for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0u, 0u, 0u, 0u);
+            if (args.lse != nullptr) args.lse[static_cast<size_t>(item.bh) * n + row_g] = -INFINITY;
+          }
+          continue;
         }
-        continue;
+        ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nfull[t] & 1, abort_flag);
+        if (ok) ok = mbar_wait_warp(smem_u32(&sm.st_full[t]), nfull[t] & 1, abort_flag);
+        if (!ok) break;
+        ++nfull[t];
+        tc_fence_after();
+        const float m = sm.stat_m[t][row];
+        float lt = sm.stat_l[t][row];
+        mbar_arrive(smem_u32(&sm.st_empty[t]));
+        // A row whose max is still -inf saw no key: its sum is only the cubic's floor
+        // for masked scores (< 1e-38 each), not probability mass.  A NaN sum marks a
+        // NaN input: the row comes out NaN.
+        if (OFFSET && m == -INFINITY && lt == lt) lt = 0.f;
+        const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
+        const uint32_t tO = tmem + lane_off + 256 + t * 128;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          FA_TMEM_LD32(tO + 32 * c, o);
+          tmem_ld_wait();
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&sm.o_free[t]));
+          }
+          if (row_g < n) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 w;
+              w.x = pack2<T>(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+              w.y = pack2<T>(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+              w.z = pack2<T>(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+              w.w = pack2<T>(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+              dst[v4] = w;
+            }
+          }
+        }
+        if (row_g < n && args.lse != nullptr)
+          args.lse[static_cast<size_t>(item.bh) * n + row_g] =
+              lt > 0.f ? m * args.scale + logf(lt) : (lt == 0.f ? -INFINITY : lt);
       }
-      const int row_p = row_g + geo.q_off;  // the row's position in the key sequence
-      float m = -INFINITY, l = 0.f;  // l: this thread's half of the row sum
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    // Warpgroup t is the softmax of query tile slot t: thread = row (TMEM lane
+    // 32 (warp % 4) + lane), all 128 score columns of the key tile in registers.
+    regs_inc<kSoftmaxRegs>();
+    const int t = wg;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
+    const float sl2 = args.scale_log2;
+    int ns = 0;     // S tiles consumed (s_full phase)
+    int nst = 0;    // items published (st_full / st_empty phase)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int lin = item_of(k, total);
+      if (lin < 0) break;
+      const Item item = make_item<OFFSET>(lin, BH, num_pairs, geo);
+      if (!active(item, t)) continue;  // the epilogue writes an inactive tile's rows
+      const int r0 = item.r0[t];
+      const int row_p = r0 + row + geo.q_off;  // the row's position in the key sequence
+      float m = -INFINITY, l = 0.f;
       bool nan_row = false;
       for (int j = item.lo_t[t]; j < item.hi_t[t]; ++j, ++ns) {
         ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), ns & 1, abort_flag);
+        if (!ok) break;
         tc_fence_after();
-        uint32_t s[64];
+        uint32_t s[BN];
         FA_TMEM_LD32(tS + 0, (s + 0));
         FA_TMEM_LD32(tS + 32, (s + 32));
+        FA_TMEM_LD32(tS + 64, (s + 64));
+        FA_TMEM_LD32(tS + 96, (s + 96));
         tmem_ld_wait();
-        const bool masked = tile_needs_mask(j, r0, geo);
-        if (masked) {
-          // Visible keys of this row form one interval; columns of this half are 64h + c.
-          const int base = j * BN + 64 * hc;
-          int c_hi = min(64, geo.Nk - base);
+        if (tile_needs_mask(j, r0, geo)) {
+          // Visible keys of this row form one interval of the tile's columns.
+          const int base = j * BN;
+          int c_hi = min(BN, geo.Nk - base);
           if (args.causal) c_hi = min(c_hi, row_p - base + 1);
           const int c_lo = args.window > 0 ? max(0, row_p - args.window + 1 - base) : 0;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < BN; ++c)
             if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
         }
-        // Half-row max: eight chains of 3-input max; NaN-propagating so a NaN score
-        // marks the row (its output is NaN at the end).
+        // Row max: eight chains of 3-input max; NaN-propagating so a NaN score marks
+        // the row (its output is NaN at the end).
         float mm[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           mm[q] = fmax3_nan(__uint_as_float(s[q]), __uint_as_float(s[q + 8]), -INFINITY);
 #pragma unroll
-        for (int c = 16; c < 64; c += 16)
+        for (int c = 16; c < BN; c += 16)
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             mm[q] = fmax3_nan(mm[q], __uint_as_float(s[c + q]), __uint_as_float(s[c + 8 + q]));
-        const float hm = fmax3_nan(fmax3_nan(mm[0], mm[1], mm[2]), fmax3_nan(mm[3], mm[4], mm[5]),
+        const float mx = fmax3_nan(fmax3_nan(mm[0], mm[1], mm[2]), fmax3_nan(mm[3], mm[4], mm[5]),
                                    fmax3_nan(mm[6], mm[7], -INFINITY));
-        sm.xmax[t][ns & 1][hc][row] = hm;
-        // Barrier of the tile's 256 threads: both halves' maxima are visible, and the
-        // whole group agrees on whether to go on.
-        ok = named_bar_all(ok, bar_id, kBarThreads);
-        if (!ok) break;
-        const float mx = fmax3_nan(hm, sm.xmax[t][ns & 1][hc ^ 1][row], -INFINITY);
         nan_row |= (mx != mx);
         const float m_new = fmaxf(m, mx);  // ignores a NaN mx
         // (m_new - m) is +inf on the first visible tile and NaN while the row is
-        // still empty; only the former moves the reference max.  Both halves of a
-        // row take the same decision from the same numbers.
+        // still empty; only the former moves the reference max.
         const bool need = (m_new - m) * sl2 > kRescaleThreshold;
         float alpha = 1.f;
         if (need) {
@@ -530,16 +645,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           m = m_new;
           l *= alpha;
         }
-        const float ms = (m == -INFINITY) ? 0.f : m * sl2;
-        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> 16-bit pairs over this
-        // half's first 32 S columns (already read).  Scores go in pairs through the
-        // packed f32x2 FMA; kPolyPairs of every 8 pairs take 2^x from the cubic on
-        // the FMA pipe, the rest from the special-function unit, so both pipes share
-        // the exponentials.
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), nms2 = f2_pack(-ms, -ms);
-        uint64_t acc_a = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
+        if (j > item.lo_t[t] && __any_sync(0xffffffffu, need)) {
+          // O_t's last update (PV_t(j-1)) is complete: S_t(j) was issued after it.
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            FA_TMEM_LD32(tO + 32 * c, r);
+            tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            FA_TMEM_ST32(tO + 32 * c, r);
+          }
+        }
+        const float ms = (m == -INFINITY) ? 0.f : m * sl2;
+        // P = 2^(s * scale * log2(e) - m * scale * log2(e)) -> 16-bit pairs in S columns
+        // [0, 64) (already read).  Scores go in pairs through the packed f32x2 FMA;
+        // kPolyPairs of every 8 pairs take 2^x from the cubic on the FMA pipe, the rest
+        // from the special-function unit, so both pipes share the exponentials.
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nms2 = f2_pack(-ms, -ms);
+        uint64_t acc[4] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
           uint32_t p[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
@@ -553,7 +679,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               f2_unpack(x2, x0, x1);
               p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
             }
-            if (e & 2) acc_b = f2_add(acc_b, p2); else acc_a = f2_add(acc_a, p2);
+            acc[(e >> 1) & 3] = f2_add(acc[(e >> 1) & 3], p2);
             float p0, p1;
             f2_unpack(p2, p0, p1);
             p[e >> 1] = pack2<T>(p0, p1);
@@ -565,67 +691,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               "r"(p[8]), "r"(p[9]), "r"(p[10]), "r"(p[11]), "r"(p[12]), "r"(p[13]), "r"(p[14]), "r"(p[15])
               : "memory");
         }
-        if (j > item.lo_t[t] && __any_sync(0xffffffffu, need)) {
-          // O_t's last update (PV_t(j-1)) is complete: S_t(j) was issued after it.
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r[32];
-            FA_TMEM_LD32(tO + 32 * c, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            FA_TMEM_ST32(tO + 32 * c, r);
-          }
-        }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(smem_u32(&sm.p_full[t]));
         {
-          float a0, a1, b0, b1;
-          f2_unpack(acc_a, a0, a1);
-          f2_unpack(acc_b, b0, b1);
-          l += (a0 + a1) + (b0 + b1);
+          const uint64_t s01 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+          float a0, a1;
+          f2_unpack(s01, a0, a1);
+          l += a0 + a1;
         }
       }
       if (!ok) break;
-      // Epilogue: O / l in 16 bits and lse = m * scale + ln l.  O_t is read out first and
-      // released (o_free) so the next item's PV can start while the stores drain.
-      ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nout & 1, abort_flag);
-      ++nout;
-      tc_fence_after();
-      uint32_t o[64];
-      FA_TMEM_LD32(tO + 0, (o + 0));
-      FA_TMEM_LD32(tO + 32, (o + 32));
-      tmem_ld_wait();
-      tc_fence_before();
-      sm.xsum[t][hc][row] = l;
-      ok = named_bar_all(ok, bar_id, kBarThreads);
-      mbar_arrive(smem_u32(&sm.o_free[t]));
+      // Publish the item's row statistics for the epilogue (the previous item's
+      // must have been read first).
+      if (nst > 0) ok = mbar_wait_warp(smem_u32(&sm.st_empty[t]), (nst - 1) & 1, abort_flag);
       if (!ok) break;
-      float lt = l + sm.xsum[t][hc ^ 1][row];
-      // The sums may be read again only after the next item's first exchange barrier.
-      // A row whose max is still -inf saw no key: its sum is only the cubic's floor
-      // for masked scores (< 1e-38 each), not probability mass.
-      if (OFFSET && m == -INFINITY) lt = 0.f;
-      if (nan_row) lt = __uint_as_float(0x7fc00000u);  // NaN input: NaN output row
-      const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
-      if (row_g < n) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(args.o) +
-                              (static_cast<size_t>(item.bh) * n + row_g) * D + 64 * hc;
-        uint4* dst = reinterpret_cast<uint4*>(orow);
-#pragma unroll
-        for (int v4 = 0; v4 < 8; ++v4) {
-          uint4 w;
-          w.x = pack2<T>(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
-          w.y = pack2<T>(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
-          w.z = pack2<T>(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
-          w.w = pack2<T>(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
-          dst[v4] = w;
-        }
-        if (hc == 0 && args.lse != nullptr)
-          args.lse[static_cast<size_t>(item.bh) * n + row_g] =
-              lt > 0.f ? m * args.scale + logf(lt) : (lt == 0.f ? -INFINITY : lt);
-      }
+      sm.stat_m[t][row] = m;
+      sm.stat_l[t][row] = nan_row ? __uint_as_float(0x7fc00000u) : l;
+      mbar_arrive(smem_u32(&sm.st_full[t]));
+      ++nst;
     }
   }
 
@@ -650,7 +734,13 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   const bool offset = a.q_off != 0 || a.Nk != a.N;
   auto kernel = offset ? (a.f16 ? fwd_tc_kernel<F16, true> : fwd_tc_kernel<Bf16, true>)
                        : (a.f16 ? fwd_tc_kernel<F16, false> : fwd_tc_kernel<Bf16, false>);
-  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), kSmemBytes);
+  // The register split draws on the 128 registers per thread the block is launched
+  // with; with fewer, setmaxnreg.inc would wait forever, so never launch then.
+  cudaFuncAttributes fattr{};
+  cudaError_t e = cudaFuncGetAttributes(&fattr, reinterpret_cast<const void*>(kernel));
+  if (e != cudaSuccess) return e;
+  if (fattr.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
   const long long items = static_cast<long long>((a.N + 2 * BM - 1) / (2 * BM)) * heads;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
