@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (args.window > 0) q_hi = min(32, key + args.window - qbase);
           q_hi = min(q_hi, n - qbase);  // queries past N have lse2 = +inf anyway
           if (key >= n) q_hi = 0;
+          q_hi = max(q_hi, q_lo);  // an empty interval keeps nothing
         }
         const float4* l4 = reinterpret_cast<const float4*>(&sm.lse2[s][64 * h + 32 * hc]);
         const float4* d4 = reinterpret_cast<const float4*>(&sm.delta[s][64 * h + 32 * hc]);
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int u = 0; u < 4; ++u) {
               const int e = 4 * e4 + u;
               float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lq[u]));
-              if (masked && (16 * c + e < q_lo || 16 * c + e >= q_hi)) p = 0.f;
+              if (masked) p = keep_or_zero(p, 16 * c + e, q_lo, q_hi);
               pv[u] = p;
               dsv[u] = p * (__uint_as_float(dr[e]) - dq[u]);
             }

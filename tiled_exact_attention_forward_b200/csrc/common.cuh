@@ -432,6 +432,30 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// x if lo <= c < hi, else -inf (as raw bits), without a branch: the caller's
+// bounds differ from lane to lane, and a per-element `if` there compiles to
+// divergent branches that cost far more than the compare and select.
+__device__ __forceinline__ uint32_t keep_or_ninf(uint32_t x, int c, int lo, int hi) {
+  uint32_t r;
+  asm("{\n\t.reg .pred p;\n\t"
+      "setp.lt.u32 p, %1, %2;\n\t"
+      "selp.b32 %0, %3, 0xff800000, p;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(c - lo)), "r"(static_cast<uint32_t>(hi - lo)), "r"(x));
+  return r;
+}
+
+// x if lo <= c < hi, else 0, without a branch (see keep_or_ninf).
+__device__ __forceinline__ float keep_or_zero(float x, int c, int lo, int hi) {
+  float r;
+  asm("{\n\t.reg .pred p;\n\t"
+      "setp.lt.u32 p, %1, %2;\n\t"
+      "selp.f32 %0, %3, 0f00000000, p;\n\t}"
+      : "=f"(r)
+      : "r"(static_cast<uint32_t>(c - lo)), "r"(static_cast<uint32_t>(hi - lo)), "f"(x));
+  return r;
+}
+
 // Visibility rule of the mask (see fa.h).
 __device__ __forceinline__ bool key_visible(int i, int j, int n, int causal, int window) {
   return j < n && (!causal || j <= i) && (window <= 0 || j > i - window);

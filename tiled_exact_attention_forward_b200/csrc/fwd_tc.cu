@@ -22,8 +22,9 @@
 //         per query row (= TMEM lane), all 128 score columns in registers, so
 //         the row max and sum need no exchange between threads;
 //       warpgroup 2 -- the epilogue: reads O out of TMEM, divides by the row
-//         sum, stores O (16-bit) and lse, so the softmax warps go straight on
-//         to the next item's first tile;
+//         sum, stages O (16-bit) in shared memory and writes it with TMA stores,
+//         and stores lse, so the softmax warps go straight on to the next item's
+//         first tile;
 //       warpgroup 3 -- warp 12 allocates tensor memory and issues every MMA,
 //         warp 13 streams K/V through the ring by TMA, warp 14 loads the Q
 //         tiles (each as soon as its slot frees) and prefetches the next item's
@@ -78,6 +79,7 @@ constexpr int EPI_WG = 2;            // epilogue warpgroup (warps 8-11)
 constexpr int MMA_WARP = 12;
 constexpr int TMA_WARP = 13;         // K/V stream
 constexpr int QLD_WARP = 14;         // Q tiles: loaded as soon as their slot frees
+constexpr int kEpiBar = 1;           // named barrier of the epilogue warpgroup
 constexpr int kSoftmaxRegs = 192;    // 128 scores + exp2 pipeline, no spills
 constexpr int kEpilogueRegs = 64;
 constexpr int kOtherRegs = 64;
@@ -95,6 +97,7 @@ struct Smem {
   // 1024-byte aligned by construction (the dynamic buffer is aligned at runtime).
   uint8_t q[2][TILE_BYTES];
   uint8_t kv[NS][TILE_BYTES];
+  uint8_t ostage[HALF_BYTES];  // epilogue: 64 output columns of a tile, 128-byte swizzled
   uint64_t q_full[2];
   uint64_t q_empty[2];
   uint64_t kv_full[NS];
@@ -283,7 +286,8 @@ __device__ __forceinline__ int item_of(int k, int total) {
 template <class T, bool OFFSET>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, FwdArgs args) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  FwdArgs args) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -325,6 +329,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -517,6 +522,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     regs_dec<kEpilogueRegs>();
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t stage = smem_u32(sm.ostage);
+    const bool leader = threadIdx.x == EPI_WG * WG_THREADS;  // issues the TMA stores
+    bool pending = false;  // leader: a TMA store may still be reading the staging buffer
     int nfull[2] = {0, 0};
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -539,6 +547,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ok = mbar_wait_warp(smem_u32(&sm.o_full[t]), nfull[t] & 1, abort_flag);
         if (ok) ok = mbar_wait_warp(smem_u32(&sm.st_full[t]), nfull[t] & 1, abort_flag);
+        // The four epilogue warps meet at named barriers below: decide together.
+        ok = named_bar_all(ok, kEpiBar, WG_THREADS);
         if (!ok) break;
         ++nfull[t];
         tc_fence_after();
@@ -551,26 +561,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (OFFSET && m == -INFINITY && lt == lt) lt = 0.f;
         const float inv = lt > 0.f ? 1.f / lt : (lt == 0.f ? 0.f : lt);
         const uint32_t tO = tmem + lane_off + 256 + t * 128;
+        // O / l goes out through shared memory and one TMA store per 64-column half:
+        // a thread storing its own 256-byte row to global memory touches 32 cache
+        // lines per warp instruction, and that traffic was measured to stall the
+        // softmax warps' TMEM and ex2 work at every item boundary.  The TMA store
+        // also clips the rows past N.
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          FA_TMEM_LD32(tO + 32 * c, o);
-          tmem_ld_wait();
-          if (c == D / 32 - 1) {
-            tc_fence_before();
-            mbar_arrive(smem_u32(&sm.o_free[t]));
-          }
-          if (row_g < n) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int h = 0; h < 2; ++h) {
+          // The staging buffer is free once the previous TMA store has read it.
+          if (leader && pending) bulk_wait_read0();
+          named_bar_sync(kEpiBar, WG_THREADS);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            FA_TMEM_LD32(tO + 64 * h + 32 * c, o);
+            tmem_ld_wait();
+            if (h == 1 && c == 1) {
+              tc_fence_before();
+              mbar_arrive(smem_u32(&sm.o_free[t]));
+            }
+            // 16-byte chunk cc of this row's 128 bytes sits at chunk cc ^ (row % 8)
+            // (the 128-byte swizzle the tensor map expects).
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack2<T>(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
-              w.y = pack2<T>(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
-              w.z = pack2<T>(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
-              w.w = pack2<T>(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
-              dst[v4] = w;
+              const int cc = 4 * c + v4;
+              const uint32_t dst = stage + row * 128 + ((cc ^ (row & 7)) << 4);
+              const uint32_t w0 = pack2<T>(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+              const uint32_t w1 = pack2<T>(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+              const uint32_t w2 = pack2<T>(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+              const uint32_t w3 = pack2<T>(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                           : "memory");
             }
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(kEpiBar, WG_THREADS);
+          if (leader) {
+            tma_store_3d(&tm_o, stage, 64 * h, item.r0[t], item.bh);
+            bulk_commit();
+            pending = true;
           }
         }
         if (row_g < n && args.lse != nullptr)
@@ -578,6 +607,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               lt > 0.f ? m * args.scale + logf(lt) : (lt == 0.f ? -INFINITY : lt);
       }
     }
+    if (leader && pending) bulk_wait0();  // every output store completes before exit
   } else {
     // ------------------------------------------------------------ softmax warps
     // Warpgroup t is the softmax of query tile slot t: thread = row (TMEM lane
@@ -617,9 +647,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           int c_hi = min(BN, geo.Nk - base);
           if (args.causal) c_hi = min(c_hi, row_p - base + 1);
           const int c_lo = args.window > 0 ? max(0, row_p - args.window + 1 - base) : 0;
+          c_hi = max(c_hi, c_lo);  // an empty interval keeps nothing
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < BN; ++c) s[c] = keep_or_ninf(s[c], c, c_lo, c_hi);
         }
         // Row max: eight chains of 3-input max; NaN-propagating so a NaN score marks
         // the row (its output is NaN at the end).
@@ -725,11 +755,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   using namespace fwdtc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const long long heads = static_cast<long long>(a.B) * a.H;
   if (!make_tmap_half_rows(&tq, a.q, D, a.N, heads, BM, a.f16) ||
       !make_tmap_half_rows(&tk, a.k, D, a.Nk, heads, BN, a.f16) ||
-      !make_tmap_half_rows(&tv, a.v, D, a.Nk, heads, BN, a.f16))
+      !make_tmap_half_rows(&tv, a.v, D, a.Nk, heads, BN, a.f16) ||
+      !make_tmap_half_rows(&to, a.o, D, a.N, heads, BM, a.f16))
     return cudaErrorInvalidValue;
   const bool offset = a.q_off != 0 || a.Nk != a.N;
   auto kernel = offset ? (a.f16 ? fwd_tc_kernel<F16, true> : fwd_tc_kernel<Bf16, true>)
@@ -748,7 +779,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
   e = sm_count(&sms);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, a);
+  kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tq, tk, tv, to, a);
   return cudaGetLastError();
 }
 
