@@ -15,9 +15,12 @@ key) pairs the mask allows: 4*d FLOPs per pair forward, 10*d backward;
 decode counts the bytes of the K/V rows it must read plus q and o (paged: plus
 the block-table entries it uses).
 
-Prints one JSON line (rank 0).  With --gpus N > 1 (launched by torchrun) each
-rank runs its own independent batch (weak scaling, no collective on the data
-path); value = all ranks' work / the slowest rank's time.
+Prints one JSON line (rank 0).  With --gpus N > 1 each rank runs its own
+independent batch (weak scaling, no collective on the data path); value = all
+ranks' work / the slowest rank's time.  Launched without torchrun, --gpus N > 1
+starts the N ranks itself through torch.distributed.run; it stops with an error
+(exit 2, no result line) when fewer than N GPUs are visible or when --gpus
+differs from the launcher's WORLD_SIZE.
 
 --impl reference times the float64 CPU oracle (the only other
 implementation of this method) on a bounded sample of the same workload.
@@ -64,6 +67,13 @@ def backward_flops(w) -> float:
 
 
 DECODE_KINDS = ("decode", "paged_decode")
+BYTE_KINDS = DECODE_KINDS + ("merge",)  # workloads measured in GB/s against copy bandwidth
+
+
+def merge_bytes(w) -> float:
+    """Bytes one merge reads and writes: every part's O row and lse, the merged row and lse."""
+    rows = w.B * w.H * w.N
+    return float(rows) * (w.parts * (2 * w.d + 4) + 2 * w.d + 4)
 
 
 def decode_bytes(w, seqlens) -> float:
@@ -201,6 +211,14 @@ def oracle_sample(w, budget_s=12.0):
             oracle.decode_forward(q, kc, vc, np.array([n]), w.scale)
             t_total += time.perf_counter() - t0
             units += n * w.d * 2 * 2 + 2 * w.d * 2
+        elif w.kind == "merge":
+            rows = 4096
+            o_p = torch.randn((w.parts, rows, w.d), generator=gen).to(w.dtype)
+            l_p = torch.randn((w.parts, rows), generator=gen) * 3.0
+            t0 = time.perf_counter()
+            oracle.merge_partials(o_p, l_p)
+            t_total += time.perf_counter() - t0
+            units += rows * (w.parts * (2 * w.d + 4) + 2 * w.d + 4)
         elif w.kind == "paged_decode":
             n = int(workloads.decode_seqlens(w.B, w.seqlen_lo, w.seqlen_hi, w.seed)[heads % w.B])
             nb = -(-n // w.block_size)
@@ -226,6 +244,8 @@ def oracle_sample(w, budget_s=12.0):
             units += per
         heads += 1
     rate = units / t_total
+    if w.kind == "merge":
+        return rate / 1e9, f"{heads} blocks of 4096 rows x {w.parts} parts (float64), {t_total:.1f} s"
     if w.kind in DECODE_KINDS:
         return rate / 1e9, f"{heads} of {w.B * w.H} (sequence, head) decodes, {t_total:.1f} s"
     return rate / 1e12, f"{heads} of {w.B * w.H} heads (full N x N float64 per head), {t_total:.1f} s"
@@ -266,6 +286,30 @@ def make_step(w, dev, rank=0, world=1):
         d2h = o_h.numel() * o_h.element_size() + l_h.numel() * 4
         return (step, e2e, units, "GB/s", "decode GB/s", 2, "decode_split_kernel",
                 ["decode.cu", "common.cuh", "kernels.h"], h2d, d2h)
+
+    if w.kind == "merge":
+        o_parts, lse_parts = workloads.workload_inputs(w, device=dev)
+        o = torch.empty(o_parts.shape[1:], dtype=o_parts.dtype, device=dev)
+        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=dev)
+
+        def step():
+            fa.merge(o_parts, lse_parts, out=o, lse=lse)
+
+        # End to end: the parts go up, the merged rows and lse come back.
+        h_in = [t.cpu().pin_memory() for t in (o_parts, lse_parts)]
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse)]
+
+        def e2e():
+            o_parts.copy_(h_in[0], non_blocking=True)
+            lse_parts.copy_(h_in[1], non_blocking=True)
+            fa.merge(o_parts, lse_parts, out=o, lse=lse)
+            h_out[0].copy_(o, non_blocking=True)
+            h_out[1].copy_(lse, non_blocking=True)
+
+        h2d = sum(t.numel() * t.element_size() for t in h_in)
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+        return (step, e2e, merge_bytes(w) / 1e9, "GB/s", "merge GB/s", 1, "merge_kernel",
+                ["merge.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
     if w.kind == "decode":
         q, kc, vc, seqlens = workloads.workload_inputs(w, device=dev)
@@ -339,41 +383,72 @@ def make_step(w, dev, rank=0, world=1):
             ["bwd.cu" if with_bwd else "fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
-def context_parallel_plan(w):
-    """Per rank of the ring: the key shards it computes (visible ones), in ring order."""
+def context_parallel_plan(w, world=None):
+    """Per rank of the ring: its steps with the visible key-chunk partials.
+
+    Returns (chunk length, plans) with plans[r] the ring_schedule of rank r."""
     from tiled_exact_attention_forward_b200 import context_parallel as cp
 
-    Ns = w.N // w.shards
-    return Ns, [[st for st in cp.ring_schedule(r, w.shards, Ns, w.causal, w.window) if st.visible]
-                for r in range(w.shards)]
+    world = world or w.shards
+    m = cp.n_chunks(world, w.balanced)
+    if w.N % m:
+        raise ValueError(f"{w.name}: N = {w.N} does not split into {m} equal chunks")
+    C = w.N // m
+    return C, [cp.ring_schedule(r, world, C, w.causal, w.window, w.balanced) for r in range(world)]
+
+
+def ring_launches_per_step(w, world: int) -> int:
+    """Kernel launches of the whole job per ring step: every rank's visible key-chunk
+    partials plus one merge per query chunk that has more than one partial."""
+    from tiled_exact_attention_forward_b200 import context_parallel as cp
+
+    _, plans = context_parallel_plan(w, world)
+    total = 0
+    for r, plan in enumerate(plans):
+        counts = [0] * len(cp.rank_chunks(r, world, w.balanced))
+        for st in plan:
+            for p in st.partials:
+                counts[p.q_chunk] += 1
+        total += sum(counts) + sum(c > 1 for c in counts)
+    return total
 
 
 def context_parallel_emulated(w, dev, fa):
-    """All ranks of the ring on one device: each rank's sequence shard of q, k, v,
-    the key-shard partials it computes and the merge.  The exchange itself (NCCL
+    """All ranks of the ring on one device: each rank's chunks of q, k, v, the
+    key-chunk partials it computes and the merges.  The exchange itself (NCCL
     send/receive between GPUs) is not part of it: one GPU has no peer.
-    Returns (step, shards (q, k, v lists), results (o, lse lists), launches)."""
+    Returns (step, inputs (q, k, v chunk lists), results (o, lse chunk lists), launches)."""
+    from tiled_exact_attention_forward_b200 import context_parallel as cp
+
     q, k, v = workloads.workload_inputs(w, device=dev)
-    Ns, plans = context_parallel_plan(w)
-    cut = [[t[:, :, r * Ns:(r + 1) * Ns].contiguous() for r in range(w.shards)] for t in (q, k, v)]
+    C, plans = context_parallel_plan(w)
+    m = cp.n_chunks(w.shards, w.balanced)
+    cut = [[t[:, :, a * C:(a + 1) * C].contiguous() for a in range(m)] for t in (q, k, v)]
     del q, k, v
     qs, ks, vs = cut
-    o_parts = [torch.empty((len(p), w.B, w.H, Ns, w.d), dtype=w.dtype, device=dev) for p in plans]
-    l_parts = [torch.empty((len(p), w.B, w.H, Ns), dtype=torch.float32, device=dev) for p in plans]
-    merged = [len(p) > 1 for p in plans]
-    outs = [torch.empty_like(qs[r]) if merged[r] else o_parts[r][0] for r in range(w.shards)]
-    lses = [torch.empty((w.B, w.H, Ns), dtype=torch.float32, device=dev) if merged[r] else l_parts[r][0]
-            for r in range(w.shards)]
+    jobs = []  # per (rank, local query chunk): the list of (key chunk, q_offset)
+    for r, plan in enumerate(plans):
+        mine = cp.rank_chunks(r, w.shards, w.balanced)
+        for qi, a in enumerate(mine):
+            parts = [(cp.rank_chunks(st.shard, w.shards, w.balanced)[p.k_chunk], p.q_offset)
+                     for st in plan for p in st.partials if p.q_chunk == qi]
+            jobs.append((a, parts))
+    jobs.sort(key=lambda job: job[0])  # results in sequence order: chunk a of every rank
+    o_parts = [torch.empty((len(p), w.B, w.H, C, w.d), dtype=w.dtype, device=dev) for _, p in jobs]
+    l_parts = [torch.empty((len(p), w.B, w.H, C), dtype=torch.float32, device=dev) for _, p in jobs]
+    outs = [torch.empty_like(qs[a]) if len(p) > 1 else o_parts[i][0] for i, (a, p) in enumerate(jobs)]
+    lses = [torch.empty((w.B, w.H, C), dtype=torch.float32, device=dev) if len(p) > 1 else l_parts[i][0]
+            for i, (a, p) in enumerate(jobs)]
 
     def step():
-        for r, plan in enumerate(plans):
-            for i, st in enumerate(plan):
-                fa.forward_offset(qs[r], ks[st.shard], vs[st.shard], st.q_offset, w.causal, w.window,
-                                  w.scale, out=o_parts[r][i], lse=l_parts[r][i])
-            if merged[r]:
-                fa.merge(o_parts[r], l_parts[r], out=outs[r], lse=lses[r])
+        for i, (a, parts) in enumerate(jobs):
+            for n, (c, off) in enumerate(parts):
+                fa.forward_offset(qs[a], ks[c], vs[c], off, w.causal, w.window, w.scale,
+                                  out=o_parts[i][n], lse=l_parts[i][n])
+            if len(parts) > 1:
+                fa.merge(o_parts[i], l_parts[i], out=outs[i], lse=lses[i])
 
-    launches = sum(len(p) for p in plans) + sum(merged)
+    launches = sum(len(p) + (len(p) > 1) for _, p in jobs)
     return step, (qs, ks, vs), (outs, lses), launches
 
 
@@ -384,7 +459,7 @@ def _context_parallel_step(w, dev, fa):
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs + lses]
     dev_out = outs + lses
 
-    # End to end: every rank's shards go up from pinned host memory, the ring steps
+    # End to end: every rank's chunks go up from pinned host memory, the ring steps
     # run, and every rank's output rows and lse come back.
     def e2e():
         for d_, h_ in zip(dev_in, host_in):
@@ -400,42 +475,30 @@ def _context_parallel_step(w, dev, fa):
             launches, "fwd_tc_kernel", ["fwd_tc.cu", "common.cuh", "kernels.h"], h2d, d2h)
 
 
-def ring_launches_per_step(w, world: int) -> int:
-    """Kernel launches of the whole job per ring step: every rank's visible key-shard
-    partials plus one merge on each rank that has more than one partial."""
-    from tiled_exact_attention_forward_b200 import context_parallel as cp
-
-    Ns = w.N // world
-    plans = [[st for st in cp.ring_schedule(r, world, Ns, w.causal, w.window) if st.visible]
-             for r in range(world)]
-    return sum(len(p) for p in plans) + sum(len(p) > 1 for p in plans)
-
-
 def _ring_step(w, dev, fa, rank, world):
-    """The context-parallel ring across the ranks of the job: the sequence is cut into
-    `world` shards, rank r holds shard r of q, k and v, and each step is one
-    context_parallel_forward (key-shard partials, NCCL exchange of the K/V shards
-    around the ring, merge).  Every rank draws the same seeded full inputs and keeps
-    its own shard.  The total work is the whole sequence's, whatever `world` is."""
+    """The context-parallel ring across the ranks of the job: the sequence is cut
+    into chunks, rank r holds its chunks of q, k and v (r, or r and 2 world - 1 - r
+    for the balanced layout), and each step is one context_parallel_forward
+    (key-chunk partials, NCCL exchange of the K/V shards around the ring, merges).
+    Every rank draws the same seeded full inputs and keeps its own rows.  The total
+    work is the whole sequence's, whatever `world` is."""
     from tiled_exact_attention_forward_b200 import context_parallel as cp
 
-    if w.N % world:
-        raise ValueError(f"{w.name}: N = {w.N} does not split into {world} equal shards")
-    Ns = w.N // world
     q, k, v = workloads.workload_inputs(w, device=dev)
-    qs, ks, vs = (t[:, :, rank * Ns:(rank + 1) * Ns].contiguous() for t in (q, k, v))
+    qs, ks, vs = (cp.shard_rows(t, rank, world, w.balanced).contiguous() for t in (q, k, v))
     del q, k, v
     out = {}
 
     def step():
-        out["o"], out["lse"] = cp.context_parallel_forward(qs, ks, vs, w.causal, w.window, w.scale)
+        out["o"], out["lse"] = cp.context_parallel_forward(qs, ks, vs, w.causal, w.window, w.scale,
+                                                           balanced=w.balanced)
 
     host_in = [t.cpu().pin_memory() for t in (qs, ks, vs)]
     step()
     torch.cuda.synchronize(dev)
     host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out["o"], out["lse"])]
 
-    # End to end: this rank's shards go up from pinned host memory, the ring runs, and
+    # End to end: this rank's rows go up from pinned host memory, the ring runs, and
     # its output rows and lse come back.
     def e2e():
         for d_, h_ in zip((qs, ks, vs), host_in):
@@ -540,9 +603,11 @@ def run_gpu(args, rank, world, local_rank):
                                    f"replicas x{world}" if world > 1 else "single GPU"),
                    "l2": "flushed between timed steps (256 MiB write, untimed)",
                    **({"block_size": w.block_size} if w.block_size else {}),
-                   **({"shards": world, "ring": "one shard per GPU, NCCL exchange inside the timed steps"}
+                   **({"shards": world, "layout": "balanced" if w.balanced else "contiguous",
+                       "ring": "one shard per GPU, NCCL exchange inside the timed steps"}
                       if ring else
-                      {"shards": w.shards, "ring": "every rank's steps on one GPU, exchange not timed"}
+                      {"shards": w.shards, "layout": "balanced" if w.balanced else "contiguous",
+                       "ring": "every rank's steps on one GPU, exchange not timed"}
                       if w.shards else {})},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -575,9 +640,9 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append(v)
             samples.append(sample)
-    unit = "GB/s" if w.kind in DECODE_KINDS else "TFLOP/s"
+    unit = "GB/s" if w.kind in BYTE_KINDS else "TFLOP/s"
     value = float(np.mean(vals))
-    metric = {"decode": "decode GB/s", "paged_decode": "decode GB/s",
+    metric = {"decode": "decode GB/s", "paged_decode": "decode GB/s", "merge": "merge GB/s",
               "forward_backward": "attention TFLOP/s (fwd+bwd, unmasked FLOPs)"} \
         .get(w.kind, "attention TFLOP/s (fwd, unmasked FLOPs)")
     return {
@@ -587,7 +652,8 @@ def run_reference(args):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                    "window": w.window,
                    **({"block_size": w.block_size} if w.block_size else {}),
-                   **({"shards": w.shards, "ring": "the oracle takes the whole sequence at once (same result)"}
+                   **({"shards": w.shards, "layout": "balanced" if w.balanced else "contiguous",
+                       "ring": "the oracle takes the whole sequence at once (same result)"}
                       if w.shards else {})},
         "cpu_baseline": {"kind": "oracle", "value": value, "unit": unit, "cores": cpu_threads_used(),
                          "sample": samples[-1] if samples else ""},
@@ -613,11 +679,21 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    launched = "WORLD_SIZE" in os.environ
 
     if args.impl == "reference":
+        # The CPU oracle runs on rank 0 only; other ranks exit without work.
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
-        return
+        return 0
+
+    problem = launch_problem(args.gpus, world if launched else None, gpu_count())
+    if problem:
+        print(f"bench.py: {problem}", file=sys.stderr, flush=True)
+        return 2
+    if not launched and args.gpus > 1:
+        # One process per GPU: start the ranks ourselves (the same command line).
+        return subprocess.call(torchrun_command(args.gpus, sys.argv[1:]))
 
     if world > 1:
         import datetime
@@ -636,7 +712,37 @@ def main():
             import torch.distributed as tdist
 
             tdist.destroy_process_group()
+    return 0
+
+
+def gpu_count() -> int:
+    return torch.cuda.device_count() if torch.cuda.is_available() else 0
+
+
+def launch_problem(gpus: int, world_env, n_devices: int):
+    """Why this launch cannot run (a message), or None.
+
+    gpus: --gpus; world_env: WORLD_SIZE when launched by torchrun, else None;
+    n_devices: CUDA devices visible to this process."""
+    if gpus < 1:
+        return f"--gpus must be >= 1, got {gpus}"
+    if world_env is not None and world_env != gpus:
+        return f"--gpus {gpus} does not match the launcher's WORLD_SIZE {world_env}"
+    if world_env is None and gpus > n_devices:
+        return f"--gpus {gpus} needs {gpus} CUDA devices, {n_devices} visible"
+    return None
+
+
+def torchrun_command(gpus: int, argv):
+    """The command that runs this script once per GPU on this node."""
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

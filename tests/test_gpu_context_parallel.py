@@ -134,34 +134,38 @@ def test_merge_propagates_nan():
     assert torch.isfinite(o[0, 0, :3].float()).all() and torch.isfinite(lse[0, 0, 4:]).all()
 
 
-def _emulated_ring(q, k, v, G, causal, window):
+def _emulated_ring(q, k, v, G, causal, window, balanced):
     """Every rank's ring steps on this device, with the driver's own schedule."""
     B, H, N, d = q.shape
-    Ns = N // G
-    outs = []
+    m = cp.n_chunks(G, balanced)
+    C = N // m
+    chunks = [[t[:, :, a * C:(a + 1) * C].contiguous() for a in range(m)] for t in (q, k, v)]
+    res = {}
     for r in range(G):
-        sl = slice(r * Ns, (r + 1) * Ns)
-        parts = [st for st in cp.ring_schedule(r, G, Ns, causal, window) if st.visible]
-        o_p = torch.empty((len(parts), B, H, Ns, d), dtype=q.dtype, device="cuda")
-        l_p = torch.empty((len(parts), B, H, Ns), dtype=torch.float32, device="cuda")
-        for i, st in enumerate(parts):
-            ks = slice(st.shard * Ns, (st.shard + 1) * Ns)
-            fa.forward_offset(q[:, :, sl].contiguous(), k[:, :, ks].contiguous(), v[:, :, ks].contiguous(),
-                              st.q_offset, causal=causal, window=window, out=o_p[i], lse=l_p[i])
-        outs.append(fa.merge(o_p, l_p) if len(parts) > 1 else (o_p[0], l_p[0]))
+        plan = cp.ring_schedule(r, G, C, causal, window, balanced)
+        for qi, a in enumerate(cp.rank_chunks(r, G, balanced)):
+            parts = [(cp.rank_chunks(st.shard, G, balanced)[p.k_chunk], p.q_offset)
+                     for st in plan for p in st.partials if p.q_chunk == qi]
+            o_p = torch.empty((len(parts), B, H, C, d), dtype=q.dtype, device="cuda")
+            l_p = torch.empty((len(parts), B, H, C), dtype=torch.float32, device="cuda")
+            for i, (c, off) in enumerate(parts):
+                fa.forward_offset(chunks[0][a], chunks[1][c], chunks[2][c], off, causal=causal, window=window,
+                                  out=o_p[i], lse=l_p[i])
+            res[a] = fa.merge(o_p, l_p) if len(parts) > 1 else (o_p[0], l_p[0])
     torch.cuda.synchronize()
     assert fa.device_status() == fa.FA_OK
-    return torch.cat([o for o, _ in outs], dim=2), torch.cat([l for _, l in outs], dim=2)
+    return torch.cat([res[a][0] for a in range(m)], dim=2), torch.cat([res[a][1] for a in range(m)], dim=2)
 
 
-@pytest.mark.parametrize("G", [2, 4])
+@pytest.mark.parametrize("G,balanced", [(2, False), (4, False), (2, True), (4, True)])
 @pytest.mark.parametrize("causal,window", [(True, 0), (True, 300), (False, 0), (False, 200), (True, 1)])
-def test_emulated_ring_matches_full_forward(G, causal, window):
+def test_emulated_ring_matches_full_forward(G, balanced, causal, window):
     q, k, v = workloads.forward_inputs(2, 3, 1024, 128, torch.bfloat16, seed=G + window, device="cpu")
-    o, lse = _emulated_ring(q.cuda(), k.cuda(), v.cuda(), G, causal, window)
+    o, lse = _emulated_ring(q.cuda(), k.cuda(), v.cuda(), G, causal, window, balanced)
     O_ref, lse_ref = oracle.attention_forward(q, k, v, None, causal, window)
-    assert_output_close(o, O_ref, f"ring G={G} causal={causal} window={window}")
-    assert_lse_close(lse, lse_ref, f"ring lse G={G} causal={causal} window={window}")
+    what = f"ring G={G} balanced={balanced} causal={causal} window={window}"
+    assert_output_close(o, O_ref, what)
+    assert_lse_close(lse, lse_ref, what)
 
 
 def test_context_parallel_forward_without_process_group_is_forward():
@@ -173,8 +177,9 @@ def test_context_parallel_forward_without_process_group_is_forward():
 
 
 def test_full_size_context_parallel_workload_sampled():
-    """The benchmark's 16K causal context in 4 shards, in the launch configuration
-    the benchmark times; sampled rows of sampled heads against the oracle."""
+    """The benchmark's 16K causal context over 4 ring ranks (balanced layout: 8 chunks),
+    in the launch configuration the benchmark times; sampled rows of sampled heads
+    against the oracle."""
     sys.path.insert(0, ROOT)
     import bench
 
@@ -186,8 +191,8 @@ def test_full_size_context_parallel_workload_sampled():
     q, k, v = (torch.cat(t, dim=2) for t in (qs, ks, vs))
     o, lse = torch.cat(outs, dim=2), torch.cat(lses, dim=2)
     rng = np.random.default_rng(1)
-    Ns = w.N // w.shards
-    fixed = [0, 1, Ns - 1, Ns, Ns + 1, 2 * Ns + 127, 3 * Ns - 1, 3 * Ns, w.N - 1]
+    C = w.N // cp.n_chunks(w.shards, w.balanced)  # chunk boundaries are where the partials meet
+    fixed = [0, 1, C - 1, C, C + 1, 2 * C + 127, 3 * C - 1, 3 * C, 5 * C, w.N - C, w.N - 1]
     rows = np.unique(np.concatenate([fixed, rng.integers(0, w.N, 16)]))
     for h in (0, w.H // 2, w.H - 1):
         O_ref, lse_ref = oracle.attention_forward_rows(q[0, h].cpu(), k[0, h].cpu(), v[0, h].cpu(), rows,
@@ -195,3 +200,44 @@ def test_full_size_context_parallel_workload_sampled():
         assert_output_close(o[0, h][rows], O_ref, f"context parallel O head {h}")
         assert_lse_close(lse[0, h][rows], lse_ref, f"context parallel lse head {h}")
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("S", [3, 5, 8, 9])
+def test_merge_empty_parts_never_leak(S):
+    """Parts with lse = -inf are not part of the result, whatever their O holds
+    (here NaN and inf), across the kernel's batches of four parts."""
+    B, H, N, d = 1, 2, 200, 128
+    g = torch.Generator().manual_seed(40 + S)
+    o_parts = torch.randn((S, B, H, N, d), generator=g).to(torch.bfloat16)
+    lse_parts = (torch.randn((S, B, H, N), generator=g) * 4).float()
+    for s in range(0, S, 2):  # every other part empty for a third of the rows
+        lse_parts[s, :, :, s % 3::3] = -float("inf")
+        o_parts[s, :, :, s % 3::3] = float("nan") if s % 4 == 0 else float("inf")
+    lse_parts[:, 0, 1, 7] = -float("inf")  # one row no part saw
+    o, lse = fa.merge(o_parts.cuda(), lse_parts.cuda())
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    clean = torch.where(torch.isneginf(lse_parts)[..., None], torch.zeros_like(o_parts), o_parts)
+    O_ref, lse_ref = oracle.merge_partials(clean, lse_parts)
+    assert torch.isfinite(o.float()).all()
+    assert torch.all(o[0, 1, 7] == 0) and torch.isneginf(lse[0, 1, 7])
+    assert_output_close(o, O_ref, f"merge S={S} with empty parts")
+    live = np.isfinite(lse_ref)
+    assert_lse_close(lse.cpu()[torch.from_numpy(live)], lse_ref[live], f"merge lse S={S}")
+
+
+@pytest.mark.parametrize("name", ["merge_parts_2", "merge_parts_4", "merge_parts_8"])
+def test_full_size_merge_workload_sampled(name):
+    """The merge benchmark workloads at full size, in the benchmark's launch
+    configuration; the oracle merges sampled rows."""
+    w = workloads.WORKLOADS[name]
+    o_parts, lse_parts = workloads.workload_inputs(w, device="cuda")
+    o, lse = fa.merge(o_parts, lse_parts)
+    torch.cuda.synchronize()
+    assert fa.device_status() == fa.FA_OK
+    rows = np.unique(np.concatenate([[0, 1, w.N - 1], np.random.default_rng(5).integers(0, w.N, 64)]))
+    for h in (0, w.H - 1):
+        O_ref, lse_ref = oracle.merge_partials(o_parts[:, 0, h, rows].cpu(), lse_parts[:, 0, h, rows].cpu())
+        assert_output_close(o[0, h, rows], O_ref, f"{name} O head {h}")
+        assert_lse_close(lse[0, h, rows], lse_ref, f"{name} lse head {h}")
+    assert torch.isfinite(o.float()).all()

@@ -120,3 +120,34 @@ def test_bench_line_names_the_workload_dtype():
     assert bench.dtype_name(W["causal_prefill"].dtype) == "bf16"
     assert bench.dtype_name(W["causal_prefill_fp16"].dtype) == "f16"
     assert bench.dtype_name(W["single_head_fp32"].dtype) == "f32"
+
+
+def test_bench_launch_checks():
+    import bench
+
+    assert "needs 1 CUDA devices" in bench.launch_problem(1, None, 0)
+    assert bench.launch_problem(2, None, 8) is None
+    assert bench.launch_problem(2, 2, 8) is None
+    assert "WORLD_SIZE" in bench.launch_problem(2, 3, 8)
+    assert "needs 2 CUDA devices" in bench.launch_problem(2, None, 1)
+    assert bench.launch_problem(0, None, 8) is not None
+    cmd = bench.torchrun_command(4, ["--gpus", "4", "--steps", "2"])
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=4" in cmd
+    assert "--master-addr=127.0.0.1" in cmd and cmd[-3:] == ["4", "--steps", "2"]
+
+
+def test_bench_multi_gpu_request_without_gpus_fails_cleanly():
+    """On a machine without enough GPUs, --gpus 2 must not print a one-GPU result."""
+    import subprocess
+    import sys
+
+    import torch
+
+    if torch.cuda.is_available() and torch.cuda.device_count() >= 2:
+        pytest.skip("this machine has two GPUs")
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "1"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 2, (r.returncode, r.stderr[-2000:])
+    assert r.stdout.strip() == ""
+    assert "needs 2 CUDA devices" in r.stderr

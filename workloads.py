@@ -43,6 +43,8 @@ class Workload:
     seqlen_hi: int = 0
     block_size: int = 0  # paged decode only: rows per cache block
     shards: int = 0      # context parallel only: sequence shards (ranks of the ring)
+    balanced: bool = False  # context parallel only: rank r holds chunks r and 2 shards - 1 - r
+    parts: int = 0       # merge only: partial results merged per row
     notes: str = field(default="", compare=False)
 
     @property
@@ -71,10 +73,18 @@ WORKLOADS = {
                  seqlen_lo=512, seqlen_hi=8192, block_size=16,
                  notes="single-token decode against a paged cache: 16-row blocks, "
                        "shuffled in one pool, the lengths of kv_cache_decode"),
+        Workload("merge_parts_2", "merge", 1, 32, 16384, 128, BF16, 6, parts=2,
+                 notes="merge of 2 partial results per row (the context-parallel combine), "
+                       "524288 rows of d = 128"),
+        Workload("merge_parts_4", "merge", 1, 16, 16384, 128, BF16, 6, parts=4,
+                 notes="merge of 4 partial results per row, 262144 rows of d = 128"),
+        Workload("merge_parts_8", "merge", 1, 8, 16384, 128, BF16, 6, parts=8,
+                 notes="merge of 8 partial results per row, 131072 rows of d = 128"),
         Workload("context_parallel_causal", "context_parallel", 1, 32, 16384, 128, BF16, 5,
-                 causal=True, shards=4,
-                 notes="causal forward of a 16K context cut into 4 sequence shards: every "
-                       "rank's ring steps (key-shard partials, then the merge) run on one GPU"),
+                 causal=True, shards=4, balanced=True,
+                 notes="causal forward of a 16K context over 4 ring ranks, each holding sequence "
+                       "chunks r and 7 - r of 8 (equal causal work per rank); on one GPU every "
+                       "rank's ring steps (key-chunk partials, then the merges) run in turn"),
     ]
 }
 
@@ -169,11 +179,22 @@ def paged_decode_inputs(B, H, block_size, max_blocks, d, lo, hi, dtype=BF16, see
     return q, kpool, vpool, table.to(device), seqlens.to(device)
 
 
+def merge_inputs(S, B, H, N, d, dtype=BF16, seed=0, device="cpu"):
+    """o_parts [S, B, H, N, d] (N(0,1) rounded to dtype) and lse_parts [S, B, H, N]
+    float32 (3 N(0,1), so the parts' weights differ widely)."""
+    g = _gen(seed, device)
+    o_parts = randn((S, B, H, N, d), dtype, g, device)
+    lse_parts = randn((S, B, H, N), torch.float32, g, device) * 3.0
+    return o_parts, lse_parts
+
+
 def workload_inputs(w: Workload, device="cpu", **kw):
     """Inputs of a named workload at its full size."""
     if w.kind == "decode":
         return decode_inputs(w.B, w.H, w.N, w.d, w.seqlen_lo, w.seqlen_hi, w.dtype,
                              w.seed, device, **kw)
+    if w.kind == "merge":
+        return merge_inputs(w.parts, w.B, w.H, w.N, w.d, w.dtype, w.seed, device)
     if w.kind == "paged_decode":
         return paged_decode_inputs(w.B, w.H, w.block_size, w.N // w.block_size, w.d, w.seqlen_lo,
                                    w.seqlen_hi, w.dtype, w.seed, device, **kw)
