@@ -79,40 +79,75 @@ __device__ __forceinline__ bool tile_needs_mask(int kt, int qi, int n, int causa
   return (k1 >= n) || (causal && q0 < k1) || (window > 0 && q1 - k0 >= window);
 }
 
+// The MMA warp runs warp-uniformly and one elected lane issues each MMA and
+// commit; descriptor offsets are immediates added inside the asm.  (A single
+// thread issues tcgen05.mma barely faster than the tensor core retires a
+// 128 x 128 x 16 step, and a warp branching with one active lane issues slower
+// still -- measured on the forward.)
+template <uint32_t OFF_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
+__device__ __forceinline__ void mma_ss_e(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t acc_in) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
+      "add.s64 ad, %1, %4;\n\t"
+      "add.s64 bd, %2, %5;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %6, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(OFF_A), "n"(OFF_B), "n"(IDESC)
+      : "memory");
+}
+template <uint32_t COL_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
+__device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t acc_in) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b32 at;\n\t.reg .b64 bd;\n\t"
+      "add.u32 at, %1, %4;\n\t"
+      "add.s64 bd, %2, %5;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %6, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(COL_A), "n"(OFF_B), "n"(IDESC)
+      : "memory");
+}
+__device__ __forceinline__ void commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+// 128-byte-swizzled descriptor with the given leading-byte offset (stride 1024).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo) { return smem_desc_sw128(saddr, lbo, 1024); }
+
 // A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
-template <class T>
-__device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+template <class T, int KK = 0>
+__device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc) {
+  constexpr uint32_t off = ((KK >> 2) * HALF_BYTES + (KK & 3) * 32) >> 4, acc = KK > 0 ? 1u : 0u;
   constexpr uint32_t idesc = idesc_f32acc<T>(128, 128, 0, 0);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-    mma_ss(d_tmem, smem_desc_sw128(a_smem + off, 16, 1024), smem_desc_sw128(b_smem + off, 16, 1024),
-           idesc, kk > 0 ? 1u : 0u);
-  }
+  mma_ss_e<off, off, idesc, acc>(d_tmem, a_desc, b_desc, 0u);
+  if constexpr (KK + 1 < D / 16) issue_abT<T, KK + 1>(d_tmem, a_desc, b_desc);
 }
 
 // D[128 x d] (+)= A[tmem, 128 keys x 64 queries of half H, 16-bit] * B, B = [128 rows (K)][d]
 // tile (MN-major), rows 64H .. 64H + 63.  The A columns of queries [16k, 16k + 16) sit at
 // TMEM columns 64 (k / 4) + 32 ((k % 4) / 2) + 8 (k % 2) (16-bit pairs), where the P/dS
 // thread that owns those queries wrote them over S^T / dP^T columns it had read.
-template <int H, class T>
-__device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem,
-                                                   bool accumulate) {
+template <int H, class T, int I = 0>
+__device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                   uint32_t accumulate) {
+  constexpr int kk = 4 * H + I;
+  constexpr uint32_t col = (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8;
+  constexpr uint32_t off = (kk * 2048) >> 4, acc = kk > 0 ? 1u : 0u;
   constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 0, 1);
-#pragma unroll
-  for (int kk = 4 * H; kk < 4 * H + 4; ++kk)
-    mma_ts(d_tmem, a_tmem + (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8,
-           smem_desc_sw128(b_smem + kk * 2048, HALF_BYTES, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  mma_ts_e<col, off, idesc, acc>(d_tmem, a_tmem, b_desc, accumulate);
+  if constexpr (I + 1 < 4) issue_tmemA_b_half<H, T, I + 1>(d_tmem, a_tmem, b_desc, accumulate);
 }
 
 // dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem).
-template <class T>
-__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_smem, uint32_t k_smem) {
+template <class T, int KK = 0>
+__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint64_t ds_desc, uint64_t k_desc) {
+  constexpr uint32_t off = (KK * 2048) >> 4, acc = KK > 0 ? 1u : 0u;
   constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 1, 1);
-#pragma unroll
-  for (int kk = 0; kk < BM / 16; ++kk)
-    mma_ss(d_tmem, smem_desc_sw128(ds_smem + kk * 2048, HALF_BYTES, 1024),
-           smem_desc_sw128(k_smem + kk * 2048, HALF_BYTES, 1024), idesc, kk > 0 ? 1u : 0u);
+  mma_ss_e<off, off, idesc, acc>(d_tmem, ds_desc, k_desc, 0u);
+  if constexpr (KK + 1 < BM / 16) issue_dq<T, KK + 1>(d_tmem, ds_desc, k_desc);
 }
 
 // T: the 16-bit type of Q, K, V, dO, P, dS and the gradients (Bf16 or F16).
@@ -193,50 +228,56 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_wait_drain(smem_u32(&sm.qdo_full[idx & 1]), (idx >> 1) & 1);
     }
   } else if (warp == MMA_WARP) {
-    if (lane == 0 && nq > 0) {
-      const uint32_t ks = smem_u32(sm.k), vs = smem_u32(sm.v), dss = smem_u32(sm.ds);
-      bool ok = mbar_wait(smem_u32(&sm.kv_full), 0, abort_flag);
-      if (ok) ok = mbar_wait(smem_u32(&sm.qdo_full[0]), 0, abort_flag);
+    // Warp-uniform loop; MMAs and commits from one elected lane.  Waits on the K/V
+    // and (Q, dO) barriers need no tcgen05 fence (TMA data); waits on barriers the
+    // P/dS and dQ warps arrive on (after their tcgen05 loads/stores) do.
+    if (nq > 0) {
+      const uint64_t kd = desc_sw128(smem_u32(sm.k), 16), vd = desc_sw128(smem_u32(sm.v), 16);
+      const uint64_t dsd = desc_sw128(smem_u32(sm.ds), HALF_BYTES), kmn = desc_sw128(smem_u32(sm.k), HALF_BYTES);
+      auto qd = [&](int s) { return desc_sw128(smem_u32(sm.q[s]), 16); };
+      auto dod = [&](int s) { return desc_sw128(smem_u32(sm.dout[s]), 16); };
+      auto qmn = [&](int s) { return desc_sw128(smem_u32(sm.q[s]), HALF_BYTES); };
+      auto domn = [&](int s) { return desc_sw128(smem_u32(sm.dout[s]), HALF_BYTES); };
+      bool ok = mbar_wait_warp(smem_u32(&sm.kv_full), 0, abort_flag);
+      if (ok) ok = mbar_wait_warp(smem_u32(&sm.qdo_full[0]), 0, abort_flag);
       if (ok) {
-        tc_fence_after();
-        issue_abT<T>(tmem + T_S, ks, smem_u32(sm.q[0]));
-        tc_commit(smem_u32(&sm.s_full));
-        issue_abT<T>(tmem + T_DP, vs, smem_u32(sm.dout[0]));
-        tc_commit(smem_u32(&sm.dp_full));
+        issue_abT<T>(tmem + T_S, kd, qd(0));
+        commit_elect(smem_u32(&sm.s_full));
+        issue_abT<T>(tmem + T_DP, vd, dod(0));
+        commit_elect(smem_u32(&sm.dp_full));
       }
       for (int idx = 0; ok && idx < nq; ++idx) {
         const int s = idx & 1;
         // dV and dK for query half 0 as soon as its P^T and dS^T are in TMEM (they run
         // while the P/dS warps work on half 1), then half 1 (two ds_ready phases per
         // query tile: parity 0, then 1).
-        ok = mbar_wait(smem_u32(&sm.ds_ready), 0, abort_flag);
+        ok = mbar_wait_warp(smem_u32(&sm.ds_ready), 0, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_tmemA_b_half<0, T>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), idx > 0);
-        issue_tmemA_b_half<0, T>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), idx > 0);
-        ok = mbar_wait(smem_u32(&sm.ds_ready), 1, abort_flag);
+        issue_tmemA_b_half<0, T>(tmem + T_DV, tmem + T_S, domn(s), idx > 0 ? 1u : 0u);
+        issue_tmemA_b_half<0, T>(tmem + T_DK, tmem + T_DP, qmn(s), idx > 0 ? 1u : 0u);
+        ok = mbar_wait_warp(smem_u32(&sm.ds_ready), 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        issue_tmemA_b_half<1, T>(tmem + T_DV, tmem + T_S, smem_u32(sm.dout[s]), true);
-        issue_tmemA_b_half<1, T>(tmem + T_DK, tmem + T_DP, smem_u32(sm.q[s]), true);
-        tc_commit(smem_u32(&sm.qdo_empty[s]));
-        issue_dq<T>(tmem + T_S, dss, ks);
-        tc_commit(smem_u32(&sm.dq_full));
+        issue_tmemA_b_half<1, T>(tmem + T_DV, tmem + T_S, domn(s), 1u);
+        issue_tmemA_b_half<1, T>(tmem + T_DK, tmem + T_DP, qmn(s), 1u);
+        commit_elect(smem_u32(&sm.qdo_empty[s]));
+        issue_dq<T>(tmem + T_S, dsd, kmn);
+        commit_elect(smem_u32(&sm.dq_full));
         if (idx + 1 < nq) {
           const int s1 = (idx + 1) & 1;
-          ok = mbar_wait(smem_u32(&sm.qdo_full[s1]), ((idx + 1) >> 1) & 1, abort_flag);
+          ok = mbar_wait_warp(smem_u32(&sm.qdo_full[s1]), ((idx + 1) >> 1) & 1, abort_flag);
+          if (!ok) break;
+          issue_abT<T>(tmem + T_DP, vd, dod(s1));
+          commit_elect(smem_u32(&sm.dp_full));
+          ok = mbar_wait_warp(smem_u32(&sm.dq_free), idx & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          issue_abT<T>(tmem + T_DP, vs, smem_u32(sm.dout[s1]));
-          tc_commit(smem_u32(&sm.dp_full));
-          ok = mbar_wait(smem_u32(&sm.dq_free), idx & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_abT<T>(tmem + T_S, ks, smem_u32(sm.q[s1]));
-          tc_commit(smem_u32(&sm.s_full));
+          issue_abT<T>(tmem + T_S, kd, qd(s1));
+          commit_elect(smem_u32(&sm.s_full));
         }
       }
-      tc_commit(smem_u32(&sm.acc_done));
+      commit_elect(smem_u32(&sm.acc_done));
       mbar_wait_drain(smem_u32(&sm.acc_done), 0);
     }
     __syncwarp();

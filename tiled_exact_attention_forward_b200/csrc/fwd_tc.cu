@@ -635,22 +635,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = mbar_wait_warp(smem_u32(&sm.s_full[t]), ns & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
+        if (tile_needs_mask(j, r0, geo)) {
+          // Visible keys of this row form one interval [c_lo, c_hi) of the tile's
+          // columns.  The mask is applied in tensor memory, 32 columns at a time in a
+          // rolled loop, before the single pass below reads S: rarely run code must
+          // stay small (an unrolled 128-column mask in the main pass was measured to
+          // cost over a thousand cycles of instruction fetch on each edge tile).
+          const int base = j * BN;
+          int c_hi = min(BN, geo.Nk - base);
+          if (geo.causal) c_hi = min(c_hi, row_p - base + 1);
+          const int c_lo = geo.window > 0 ? max(0, row_p - geo.window + 1 - base) : 0;
+          c_hi = max(c_hi, c_lo);  // an empty interval keeps nothing
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            // Chunks that every row of the warp sees whole need no change; chunks no
+            // row of the warp sees at all are overwritten with -inf without being
+            // read; only a chunk the mask edge crosses is selected element by element.
+            if (__all_sync(0xffffffffu, c_lo <= 32 * c && c_hi >= 32 * c + 32)) continue;
+            uint32_t r[32];
+            if (__all_sync(0xffffffffu, c_hi <= 32 * c || c_lo >= 32 * c + 32)) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(-INFINITY);
+            } else {
+              FA_TMEM_LD32(tS + 32 * c, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = keep_or_ninf(r[e], 32 * c + e, c_lo, c_hi);
+            }
+            FA_TMEM_ST32(tS + 32 * c, r);
+          }
+          tmem_st_wait();
+        }
         uint32_t s[BN];
         FA_TMEM_LD32(tS + 0, (s + 0));
         FA_TMEM_LD32(tS + 32, (s + 32));
         FA_TMEM_LD32(tS + 64, (s + 64));
         FA_TMEM_LD32(tS + 96, (s + 96));
         tmem_ld_wait();
-        if (tile_needs_mask(j, r0, geo)) {
-          // Visible keys of this row form one interval of the tile's columns.
-          const int base = j * BN;
-          int c_hi = min(BN, geo.Nk - base);
-          if (args.causal) c_hi = min(c_hi, row_p - base + 1);
-          const int c_lo = args.window > 0 ? max(0, row_p - args.window + 1 - base) : 0;
-          c_hi = max(c_hi, c_lo);  // an empty interval keeps nothing
-#pragma unroll
-          for (int c = 0; c < BN; ++c) s[c] = keep_or_ninf(s[c], c, c_lo, c_hi);
-        }
         // Row max: eight chains of 3-input max; NaN-propagating so a NaN score marks
         // the row (its output is NaN at the end).
         float mm[8];
