@@ -57,9 +57,9 @@
 //     when the new row max exceeds it by more than 2^8 in exp2 units; P is
 //     then at most 256, exact in the final O / l.
 //   * exp2 with scale*log2(e) folded into one packed (f32x2) FMA per score
-//     pair.  A share of the pairs takes 2^x from a cubic on the FMA pipe
-//     instead of the special-function unit, whose rate (16 results per clock
-//     per SM) otherwise equals the MMA rate for d = 128.
+//     pair, 2^x from the special-function unit (a cubic on the FMA pipe can
+//     take a share of the pairs: FA_FWD_POLY_PAIRS, off by default -- see
+//     kPolyPairs).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -88,10 +88,15 @@ static_assert(2 * WG_THREADS * kSoftmaxRegs + WG_THREADS * kEpilogueRegs + WG_TH
                   NUM_THREADS * kLaunchRegs,
               "register split exceeds the launch budget");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 8 score pairs, those exponentiated by the cubic on the FMA pipe instead
+// of the special-function unit.  With one softmax thread per row the warp is
+// bound by instruction issue, not by the ex2 unit, and the cubic only adds
+// instructions: measured on B200 (causal prefill / sliding window TFLOP/s),
+// 0 -> 727-732 / 1085, 1 -> 715 / 1071, 2 -> 707 / 1056.  Kept as a build option.
 #ifndef FA_FWD_POLY_PAIRS
-#define FA_FWD_POLY_PAIRS 1
+#define FA_FWD_POLY_PAIRS 0
 #endif
-constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;  // of every 8 score pairs, those exponentiated on the FMA pipe
+constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
 
 struct Smem {
   // 1024-byte aligned by construction (the dynamic buffer is aligned at runtime).
