@@ -192,6 +192,20 @@ def cpu_threads_used():
         return int(_CPU_THREADS)
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+
+    return platform.processor() or "unknown"
+
+
 # ----------------------------------------------------------------------------- oracle (CPU) timing
 def oracle_sample(w, budget_s=12.0):
     """Time the float64 oracle on whole heads of the workload until ~budget_s.
@@ -617,7 +631,7 @@ def run_gpu(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, sample = oracle_sample(w)
         line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cpu_threads_used(), "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "cpu": cpu_model()}
     return line
 
 
@@ -656,7 +670,7 @@ def run_reference(args):
                        "ring": "the oracle takes the whole sequence at once (same result)"}
                       if w.shards else {})},
         "cpu_baseline": {"kind": "oracle", "value": value, "unit": unit, "cores": cpu_threads_used(),
-                         "sample": samples[-1] if samples else ""},
+                         "sample": samples[-1] if samples else "", "cpu": cpu_model()},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": time.perf_counter() - t0,
     }
