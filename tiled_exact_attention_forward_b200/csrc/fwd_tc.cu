@@ -251,8 +251,23 @@ template <bool OFFSET>
 __device__ __forceinline__ Item make_item(int lin, int BH, int num_pairs, const Geom& a) {
   Item it;
   // Heaviest work first: with a causal mask the last query tiles see the most keys.
-  const int pair = num_pairs - 1 - lin / BH;
-  it.bh = lin % BH;
+  // With a causal sliding window every pair from `pf` on sees a full window (equal
+  // weight): those come first and head by head, so the CTAs in flight share the
+  // K/V of a few heads in L2 instead of the windows of every head; the lighter
+  // pairs at the start of each sequence follow, heaviest first.  Without a window
+  // pf = num_pairs and the order is pair-major over all heads.
+  const int pf = (!OFFSET && a.causal && a.window > 0) ? min(num_pairs, (a.window - 1 + 2 * BM - 1) / (2 * BM))
+                                                       : num_pairs;
+  const int nfull = num_pairs - pf;
+  int pair;
+  if (lin < BH * nfull) {
+    it.bh = lin / nfull;
+    pair = num_pairs - 1 - lin % nfull;
+  } else {
+    const int rest = lin - BH * nfull;
+    pair = pf - 1 - rest / BH;
+    it.bh = rest % BH;
+  }
   it.r0[0] = pair * 2 * BM;
   it.r0[1] = it.r0[0] + BM;
 #pragma unroll
