@@ -79,75 +79,51 @@ __device__ __forceinline__ bool tile_needs_mask(int kt, int qi, int n, int causa
   return (k1 >= n) || (causal && q0 < k1) || (window > 0 && q1 - k0 >= window);
 }
 
-// The MMA warp runs warp-uniformly and one elected lane issues each MMA and
-// commit; descriptor offsets are immediates added inside the asm.  (A single
-// thread issues tcgen05.mma barely faster than the tensor core retires a
-// 128 x 128 x 16 step, and a warp branching with one active lane issues slower
-// still -- measured on the forward.)
-template <uint32_t OFF_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
-__device__ __forceinline__ void mma_ss_e(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t acc_in) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
-      "add.s64 ad, %1, %4;\n\t"
-      "add.s64 bd, %2, %5;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %6, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(OFF_A), "n"(OFF_B), "n"(IDESC)
-      : "memory");
-}
-template <uint32_t COL_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
-__device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t acc_in) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 at;\n\t.reg .b64 bd;\n\t"
-      "add.u32 at, %1, %4;\n\t"
-      "add.s64 bd, %2, %5;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %6, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(COL_A), "n"(OFF_B), "n"(IDESC)
-      : "memory");
-}
+// The MMA warp runs warp-uniformly; each 128-deep K block of MMAs is one asm
+// statement (one elect, descriptor low words stepped by immediates: mma8_ss,
+// mma4_ts), which issues as fast as the tensor core retires them, where one asm
+// statement per MMA did not.
 __device__ __forceinline__ void commit_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
 }
-// 128-byte-swizzled descriptor with the given leading-byte offset (stride 1024).
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo) { return smem_desc_sw128(saddr, lbo, 1024); }
+// Low word of a 128-byte-swizzled descriptor (start address, leading-byte offset);
+// the high word (stride 1024, version, swizzle) is kDescHi for every tile here.
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) {
+  return static_cast<uint32_t>(smem_desc_sw128(saddr, lbo, 1024));
+}
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
 
 // A = [rows][d] tile, K-major; B = [rows][d] tile, K-major: D[128x128] = A B^T.
-template <class T, int KK = 0>
-__device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc) {
-  constexpr uint32_t off = ((KK >> 2) * HALF_BYTES + (KK & 3) * 32) >> 4, acc = KK > 0 ? 1u : 0u;
-  constexpr uint32_t idesc = idesc_f32acc<T>(128, 128, 0, 0);
-  mma_ss_e<off, off, idesc, acc>(d_tmem, a_desc, b_desc, 0u);
-  if constexpr (KK + 1 < D / 16) issue_abT<T, KK + 1>(d_tmem, a_desc, b_desc);
+template <class T>
+__device__ __forceinline__ void issue_abT(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo) {
+  constexpr uint32_t h = HALF_BYTES >> 4, idesc = idesc_f32acc<T>(128, 128, 0, 0);
+  static_assert(D / 16 == 8, "one 8-MMA block");
+  mma8_ss<idesc, 2, 4, 6, h, h + 2, h + 4, h + 6>(d_tmem, a_lo, b_lo, kDescHi, 0u);
 }
 
 // D[128 x d] (+)= A[tmem, 128 keys x 64 queries of half H, 16-bit] * B, B = [128 rows (K)][d]
 // tile (MN-major), rows 64H .. 64H + 63.  The A columns of queries [16k, 16k + 16) sit at
 // TMEM columns 64 (k / 4) + 32 ((k % 4) / 2) + 8 (k % 2) (16-bit pairs), where the P/dS
-// thread that owns those queries wrote them over S^T / dP^T columns it had read.
-template <int H, class T, int I = 0>
-__device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+// thread that owns those queries wrote them over S^T / dP^T columns it had read; B's K step
+// k is 16 rows = 2 KiB on.
+template <int H, class T>
+__device__ __forceinline__ void issue_tmemA_b_half(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
                                                    uint32_t accumulate) {
-  constexpr int kk = 4 * H + I;
-  constexpr uint32_t col = (kk >> 2) * 64 + ((kk & 3) >> 1) * 32 + (kk & 1) * 8;
-  constexpr uint32_t off = (kk * 2048) >> 4, acc = kk > 0 ? 1u : 0u;
-  constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 0, 1);
-  mma_ts_e<col, off, idesc, acc>(d_tmem, a_tmem, b_desc, accumulate);
-  if constexpr (I + 1 < 4) issue_tmemA_b_half<H, T, I + 1>(d_tmem, a_tmem, b_desc, accumulate);
+  constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 0, 1), c0 = 64 * H, o0 = (4 * H * 2048) >> 4;
+  mma4_ts<idesc, c0, c0 + 8, c0 + 32, c0 + 40, o0, o0 + 128, o0 + 256, o0 + 384>(d_tmem, a_tmem, b_lo, kDescHi,
+                                                                                accumulate);
 }
 
-// dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem).
-template <class T, int KK = 0>
-__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint64_t ds_desc, uint64_t k_desc) {
-  constexpr uint32_t off = (KK * 2048) >> 4, acc = KK > 0 ? 1u : 0u;
+// dQ[128 queries x d] = dS (A, MN-major in smem) * K (B, MN-major in smem); K step k
+// is 16 rows = 2 KiB on in both.
+template <class T>
+__device__ __forceinline__ void issue_dq(uint32_t d_tmem, uint32_t ds_lo, uint32_t k_lo) {
   constexpr uint32_t idesc = idesc_f32acc<T>(128, D, 1, 1);
-  mma_ss_e<off, off, idesc, acc>(d_tmem, ds_desc, k_desc, 0u);
-  if constexpr (KK + 1 < BM / 16) issue_dq<T, KK + 1>(d_tmem, ds_desc, k_desc);
+  static_assert(BM / 16 == 8, "one 8-MMA block");
+  mma8_ss<idesc, 128, 256, 384, 512, 640, 768, 896>(d_tmem, ds_lo, k_lo, kDescHi, 0u);
 }
 
 // T: the 16-bit type of Q, K, V, dO, P, dS and the gradients (Bf16 or F16).
@@ -232,12 +208,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // and (Q, dO) barriers need no tcgen05 fence (TMA data); waits on barriers the
     // P/dS and dQ warps arrive on (after their tcgen05 loads/stores) do.
     if (nq > 0) {
-      const uint64_t kd = desc_sw128(smem_u32(sm.k), 16), vd = desc_sw128(smem_u32(sm.v), 16);
-      const uint64_t dsd = desc_sw128(smem_u32(sm.ds), HALF_BYTES), kmn = desc_sw128(smem_u32(sm.k), HALF_BYTES);
-      auto qd = [&](int s) { return desc_sw128(smem_u32(sm.q[s]), 16); };
-      auto dod = [&](int s) { return desc_sw128(smem_u32(sm.dout[s]), 16); };
-      auto qmn = [&](int s) { return desc_sw128(smem_u32(sm.q[s]), HALF_BYTES); };
-      auto domn = [&](int s) { return desc_sw128(smem_u32(sm.dout[s]), HALF_BYTES); };
+      const uint32_t kd = desc_lo(smem_u32(sm.k), 16), vd = desc_lo(smem_u32(sm.v), 16);
+      const uint32_t dsd = desc_lo(smem_u32(sm.ds), HALF_BYTES), kmn = desc_lo(smem_u32(sm.k), HALF_BYTES);
+      auto qd = [&](int s) { return desc_lo(smem_u32(sm.q[s]), 16); };
+      auto dod = [&](int s) { return desc_lo(smem_u32(sm.dout[s]), 16); };
+      auto qmn = [&](int s) { return desc_lo(smem_u32(sm.q[s]), HALF_BYTES); };
+      auto domn = [&](int s) { return desc_lo(smem_u32(sm.dout[s]), HALF_BYTES); };
       bool ok = mbar_wait_warp(smem_u32(&sm.kv_full), 0, abort_flag);
       if (ok) ok = mbar_wait_warp(smem_u32(&sm.qdo_full[0]), 0, abort_flag);
       if (ok) {

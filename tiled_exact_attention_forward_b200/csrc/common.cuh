@@ -183,6 +183,102 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- batched MMA issue
+
+// A 128-deep K block (eight kind::f16 MMAs of K = 16) from one asm statement:
+// the warp runs it uniformly, one elected lane issues, and the descriptors'
+// 32-bit low words (start address >> 4, leading-byte offset) step by
+// compile-time offsets.  Shared-memory addresses stay below 2^18, so the
+// 14-bit address field never carries into the offset field.  Issued this way
+// the MMAs keep pace with the tensor core (64.7 cycles per 128 x 128 x 16 on
+// B200); one asm statement per MMA, each with its own elect and 64-bit
+// descriptor adds, issued one every 84 cycles.
+//
+// Both operands in shared memory; A and B advance by the same offsets
+// (O1..O7, in 16-byte units).  The first MMA accumulates only if acc0 != 0.
+template <uint32_t IDESC, uint32_t O1, uint32_t O2, uint32_t O3, uint32_t O4, uint32_t O5, uint32_t O6,
+          uint32_t O7>
+__device__ __forceinline__ void mma8_ss(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a1, b1;\n\t.reg .b64 ad, bd;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "mov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t"
+      "add.u32 a1, %1, %6;\n\tadd.u32 b1, %2, %6;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %7;\n\tadd.u32 b1, %2, %7;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %8;\n\tadd.u32 b1, %2, %8;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %9;\n\tadd.u32 b1, %2, %9;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %10;\n\tadd.u32 b1, %2, %10;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %11;\n\tadd.u32 b1, %2, %11;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t"
+      "add.u32 a1, %1, %12;\n\tadd.u32 b1, %2, %12;\n\tmov.b64 ad, {a1, %3};\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(acc0), "n"(IDESC), "n"(O1), "n"(O2), "n"(O3), "n"(O4), "n"(O5),
+      "n"(O6), "n"(O7)
+      : "memory");
+}
+// A from tensor memory: A's column advances by CA per MMA, B's low word by OB
+// (16-byte units).
+template <uint32_t IDESC, uint32_t CA, uint32_t OB>
+__device__ __forceinline__ void mma8_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a1, b1;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %5, p;\n\t"
+      "add.u32 a1, %1, %6;\n\tadd.u32 b1, %2, %13;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %7;\n\tadd.u32 b1, %2, %14;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %8;\n\tadd.u32 b1, %2, %15;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %9;\n\tadd.u32 b1, %2, %16;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %10;\n\tadd.u32 b1, %2, %17;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %11;\n\tadd.u32 b1, %2, %18;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %12;\n\tadd.u32 b1, %2, %19;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(acc0), "n"(IDESC), "n"(CA), "n"(2 * CA), "n"(3 * CA), "n"(4 * CA),
+      "n"(5 * CA), "n"(6 * CA), "n"(7 * CA), "n"(OB), "n"(2 * OB), "n"(3 * OB), "n"(4 * OB), "n"(5 * OB),
+      "n"(6 * OB), "n"(7 * OB)
+      : "memory");
+}
+
+// Four kind::f16 MMAs with A from tensor memory, per-step A column offsets
+// CA0..CA3 and B low-word offsets OB0..OB3 (16-byte units); the first MMA
+// accumulates only if acc0 != 0.
+template <uint32_t IDESC, uint32_t CA0, uint32_t CA1, uint32_t CA2, uint32_t CA3, uint32_t OB0, uint32_t OB1,
+          uint32_t OB2, uint32_t OB3>
+__device__ __forceinline__ void mma4_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi, uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a1, b1;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "add.u32 a1, %1, %6;\n\tadd.u32 b1, %2, %10;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, p;\n\t"
+      "add.u32 a1, %1, %7;\n\tadd.u32 b1, %2, %11;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %8;\n\tadd.u32 b1, %2, %12;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t"
+      "add.u32 a1, %1, %9;\n\tadd.u32 b1, %2, %13;\n\tmov.b64 bd, {b1, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], bd, %5, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(acc0), "n"(IDESC), "n"(CA0), "n"(CA1), "n"(CA2), "n"(CA3), "n"(OB0),
+      "n"(OB1), "n"(OB2), "n"(OB3)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- register split
 // Move this warpgroup's per-thread register budget up or down (all four warps of
 // the warpgroup execute the same instruction).  The budgets of all warpgroups

@@ -165,41 +165,6 @@ __device__ __forceinline__ bool tile_needs_mask(int j, int r0, const Geom& a) {
 // word with no carry out of the address field.
 __device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo) { return (saddr >> 4) | ((lbo >> 4) << 16); }
 __host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo) { return (sbo >> 4) | (1u << 14) | (2u << 29); }
-__device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) {
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
-// One kind::f16 MMA with both operands in shared memory; the descriptors are
-// the bases plus compile-time offsets (in 16-byte units) added inside the asm,
-// so an unrolled chain costs a few instructions per MMA and no registers for
-// precomputed descriptors.  The whole warp executes it and one elected lane
-// issues the MMA: the issuing warp's control flow stays uniform (a warp that
-// runs its loop on one lane issues MMAs measurably slower).
-template <uint32_t OFF_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
-__device__ __forceinline__ void mma_ss_at(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t acc_in) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
-      "add.s64 ad, %1, %4;\n\t"
-      "add.s64 bd, %2, %5;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %6, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(OFF_A), "n"(OFF_B), "n"(IDESC)
-      : "memory");
-}
-// The same with A read from tensor memory at a compile-time column offset.
-template <uint32_t COL_A, uint32_t OFF_B, uint32_t IDESC, uint32_t ACC>
-__device__ __forceinline__ void mma_ts_at(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t acc_in) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t.reg .b32 at;\n\t.reg .b64 bd;\n\t"
-      "add.u32 at, %1, %4;\n\t"
-      "add.s64 bd, %2, %5;\n\t"
-      "setp.ne.b32 p, %3, 0;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %6, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(ACC ? 1u : acc_in), "n"(COL_A), "n"(OFF_B), "n"(IDESC)
-      : "memory");
-}
 
 // tcgen05.commit from one elected lane of a warp that executes it uniformly.
 __device__ __forceinline__ void commit_elect(uint32_t bar) {
@@ -211,24 +176,22 @@ __device__ __forceinline__ void commit_elect(uint32_t bar) {
 
 // S = Q K^T: Q and K tiles K-major ([64-column half][128 rows][64 cols]); a K step
 // of 16 columns is 32 bytes inside a half, the second half 16 KiB further on.
-template <class T, int KK = 0>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
-  constexpr uint32_t off = ((KK >> 2) * HALF_BYTES + (KK & 3) * 32) >> 4, acc = KK > 0 ? 1u : 0u;
-  constexpr uint32_t idesc = idesc_f32acc<T>(BM, BN, 0, 0);
-  mma_ss_at<off, off, idesc, acc>(d_tmem, q_desc, k_desc, 0u);
-  if constexpr (KK + 1 < D / 16) issue_qk<T, KK + 1>(d_tmem, q_desc, k_desc);
+template <class T>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t h = HALF_BYTES >> 4, idesc = idesc_f32acc<T>(BM, BN, 0, 0);
+  static_assert(D / 16 == 8, "one 8-MMA block per S tile");
+  mma8_ss<idesc, 2, 4, 6, h, h + 2, h + 4, h + 6>(d_tmem, desc_lo(q_addr, 16), desc_lo(k_addr, 16), desc_hi(1024), 0u);
 }
 
 // O += P V: V tile MN-major ([64-column half][128 keys][64 cols]); a K step of
 // 16 keys is 16 rows = 2 KiB.  P of keys [2c, 2c + 1] sits in S column c (16-bit
 // pairs), so the A operand of K step kk starts at column 8 kk.  The first step
 // accumulates only when `accumulate` is set (the first PV of an item overwrites O).
-template <class T, int KK = 0>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc, uint32_t accumulate) {
-  constexpr uint32_t col = KK * 8, off = (KK * 16 * 128) >> 4, acc = KK > 0 ? 1u : 0u;
-  constexpr uint32_t idesc = idesc_f32acc<T>(BM, D, 0, 1);
-  mma_ts_at<col, off, idesc, acc>(d_tmem, p_tmem, v_desc, accumulate);
-  if constexpr (KK + 1 < BN / 16) issue_pv<T, KK + 1>(d_tmem, p_tmem, v_desc, accumulate);
+template <class T>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_addr, uint32_t accumulate) {
+  static_assert(BN / 16 == 8, "one 8-MMA block per PV");
+  constexpr uint32_t idesc = idesc_f32acc<T>(BM, D, 0, 1), col_step = 8, v_step = (16 * 128) >> 4;
+  mma8_ts<idesc, col_step, v_step>(d_tmem, p_tmem, desc_lo(v_addr, HALF_BYTES), desc_hi(1024), accumulate);
 }
 
 // One unit of work: two 128-row query tiles (rows [256p, 256p + 256)) of one
@@ -448,8 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ph ^= 1u << (Q_PH + t);
             ph |= 1u << (QRDY + t);
           }
-          issue_qk<T>(tmem + 128 * t, desc_of(desc_lo(smem_u32(sm.q[t]), 16), desc_hi(1024)),
-                      desc_of(desc_lo(k_addr, 16), desc_hi(1024)));
+          issue_qk<T>(tmem + 128 * t, smem_u32(sm.q[t]), k_addr);
           commit_elect(smem_u32(&sm.s_full[t]));
           if (last) {
             commit_elect(smem_u32(&sm.q_empty[t]));
@@ -465,10 +427,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!mbar_wait_warp(smem_u32(&sm.o_free[t]), bit(O_PH + t), abort_flag)) return false;
             ph ^= 1u << (O_PH + t);
           }
-          const uint64_t vs = desc_of(desc_lo(v_addr, HALF_BYTES), desc_hi(1024));
           if (!mbar_wait_warp(smem_u32(&sm.p_full[t]), bit(PV_PH + t), abort_flag)) return false;
           tc_fence_after();
-          issue_pv<T>(tmem + 256 + 128 * t, tmem + 128 * t, vs, first ? 0u : 1u);
+          issue_pv<T>(tmem + 256 + 128 * t, tmem + 128 * t, v_addr, first ? 0u : 1u);
           ph ^= 1u << (PV_PH + t);
           if (last) {
             commit_elect(smem_u32(&sm.o_full[t]));
