@@ -142,10 +142,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int n = args.N;
   const int BH = args.B * args.H;
   const int nkt = (n + BM - 1) / BM;
-  // Causal: low key tiles see the most query tiles -> launch them first.
-  const int kt = static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  (void)nkt;
+  // CTAs go out in groups of kHeadGroup heads: within a group, low key tiles (which see
+  // the most query tiles under a causal mask) first, across the group's heads.  The
+  // CTAs in flight then cover about kHeadGroup heads, whose Q, dO and fp32 dQ
+  // accumulator stay in L2, instead of every head at once; a simulated list schedule
+  // of the causal workload keeps the same makespan as key-tile-major over all heads.
+  constexpr int kHeadGroup = 8;
+  const int g = BH < kHeadGroup ? BH : kHeadGroup;
+  const int full = BH / g, rem = BH % g;
+  const int idx = static_cast<int>(blockIdx.x);
+  int kt, bh;
+  if (idx < full * g * nkt) {
+    const int grp = idx / (g * nkt), r = idx % (g * nkt);
+    kt = r / g;
+    bh = grp * g + r % g;
+  } else {
+    const int r = idx - full * g * nkt;
+    kt = r / rem;
+    bh = full * g + r % rem;
+  }
   int qlo, qhi;
   q_tile_range(kt, n, args.causal, args.window, qlo, qhi);
   const int nq = qhi - qlo;
