@@ -70,10 +70,15 @@ DECODE_KINDS = ("decode", "paged_decode")
 BYTE_KINDS = DECODE_KINDS + ("merge",)  # workloads measured in GB/s against copy bandwidth
 
 
+def merge_row_bytes(w) -> int:
+    """Bytes per merged row: every part's O row and lse, the merged row and lse."""
+    es = torch.finfo(w.dtype).bits // 8
+    return w.parts * (es * w.d + 4) + es * w.d + 4
+
+
 def merge_bytes(w) -> float:
-    """Bytes one merge reads and writes: every part's O row and lse, the merged row and lse."""
-    rows = w.B * w.H * w.N
-    return float(rows) * (w.parts * (2 * w.d + 4) + 2 * w.d + 4)
+    """Bytes one merge reads and writes."""
+    return float(w.B * w.H * w.N) * merge_row_bytes(w)
 
 
 def decode_bytes(w, seqlens) -> float:
@@ -232,7 +237,7 @@ def oracle_sample(w, budget_s=12.0):
             t0 = time.perf_counter()
             oracle.merge_partials(o_p, l_p)
             t_total += time.perf_counter() - t0
-            units += rows * (w.parts * (2 * w.d + 4) + 2 * w.d + 4)
+            units += rows * merge_row_bytes(w)
         elif w.kind == "paged_decode":
             n = int(workloads.decode_seqlens(w.B, w.seqlen_lo, w.seqlen_hi, w.seed)[heads % w.B])
             nb = -(-n // w.block_size)

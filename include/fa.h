@@ -124,11 +124,14 @@ FA_API fa_status fa_forward_offset(const void* q, const void* k, const void* v, 
  * identity for two partial softmaxes, restated for S parts):
  *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
  *
- *   o_parts   : [S][B][H][N][d] normalised partial outputs (FA_BF16 or
- *               FA_FP16, d = 64 or 128), 16-byte aligned.
+ *   o_parts   : [S][B][H][N][d] normalised partial outputs in `dtype`:
+ *               FA_BF16, FA_FP16, or FA_FP32 (float32 partials, for callers
+ *               that keep their partials unrounded); d = 64 or 128;
+ *               16-byte aligned.
  *   lse_parts : [S][B][H][N] float32; -inf marks a part with no visible key
  *               for that row (its O is not read).
- *   o         : [B][H][N][d] output; lse: [B][H][N] float32 output or NULL.
+ *   o         : [B][H][N][d] output in `dtype`; lse: [B][H][N] float32
+ *               output or NULL.
  *   S         : 1 .. 65536.
  * A row whose parts are all empty gets O = 0 and lse = -inf; a NaN lse in any
  * part makes the row NaN.

@@ -37,9 +37,9 @@ def test_status_strings_and_version(lib):
     for code in range(5):
         assert lib.fa_status_string(code).startswith(b"FA_")
     assert lib.fa_status_string(99) == b"unknown fa_status"
-    # 1.03: fa_selftest_exp2_poly added to 1.02 (fa_forward_offset, fa_merge), which
-    # added to 1.01 (fa_decode_paged, FA_FP16).
-    assert lib.fa_version() == 103
+    # 1.04: fa_merge accepts float32 partials; 1.03 added fa_selftest_exp2_poly to
+    # 1.02 (fa_forward_offset, fa_merge), which added to 1.01 (fa_decode_paged, FA_FP16).
+    assert lib.fa_version() == 104
 
 
 P = ctypes.c_void_p
@@ -100,7 +100,8 @@ def test_merge_rejects_bad_arguments(lib):
     assert mg(parts=MISALIGNED) == fa.FA_ERR_INVALID
     assert mg(lse_parts=P(0x100002)) == fa.FA_ERR_INVALID
     assert mg(d=96) == fa.FA_ERR_UNSUPPORTED
-    assert mg(dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
+    assert mg(dtype=7) == fa.FA_ERR_UNSUPPORTED  # no such dtype (float32 partials are supported)
+    assert mg(dtype=fa.FA_FP32, d=96) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments(lib):

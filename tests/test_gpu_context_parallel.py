@@ -124,6 +124,48 @@ def test_merge_matches_oracle(dtype, d, S):
     assert_lse_close(lse.cpu()[torch.from_numpy(live)], lse_ref[live], f"merged lse S={S} d={d}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("S", [1, 2, 5, 8])
+def test_merge_float32_partials_match_oracle(d, S):
+    """float32 partials merge in float32 throughout: the result is within float32
+    rounding of the float64 merge (the 16-bit tolerances do not apply)."""
+    B, H, N = 2, 3, 257
+    g = torch.Generator().manual_seed(100 + S * d)
+    o_parts = torch.randn((S, B, H, N, d), generator=g, dtype=torch.float64)
+    lse_parts = torch.randn((S, B, H, N), generator=g, dtype=torch.float64) * 4
+    lse_parts[0, 0, 0, ::3] = -float("inf")
+    lse_parts[:, 1, 1, 10] = -float("inf")
+    o_p32, l_p32 = o_parts.float(), lse_parts.float()
+    o, lse = fa.merge(o_p32.cuda(), l_p32.cuda())
+    torch.cuda.synchronize()
+    assert o.dtype == torch.float32
+    # The oracle merges exactly the float32 values the kernel read.
+    O_ref, lse_ref = oracle.merge_partials(o_p32.double(), l_p32.double())
+    assert_output_close(o, O_ref, f"float32 merge S={S} d={d}", max_tol=5e-5, mean_tol=1e-6)
+    live = np.isfinite(lse_ref)
+    assert np.all(np.isneginf(lse.cpu().numpy()[~live]))
+    assert torch.all(o.cpu()[1, 1, 10] == 0)
+    assert_lse_close(lse.cpu()[torch.from_numpy(live)], lse_ref[live], f"float32 merge lse S={S}", tol=5e-5)
+
+
+def test_merge_float32_empty_parts_never_leak():
+    """A float32 part with lse = -inf for a row is not read into the result, even
+    when its O holds NaN there."""
+    S, B, H, N, d = 3, 1, 2, 64, 128
+    g = torch.Generator().manual_seed(7)
+    o_parts = torch.randn((S, B, H, N, d), generator=g)
+    lse_parts = torch.randn((S, B, H, N), generator=g)
+    lse_parts[1, :, :, ::2] = -float("inf")
+    o_parts[1, :, :, ::2] = float("nan")
+    o, lse = fa.merge(o_parts.cuda(), lse_parts.cuda())
+    torch.cuda.synchronize()
+    clean = o_parts.clone()
+    clean[1, :, :, ::2] = 0.0
+    O_ref, lse_ref = oracle.merge_partials(clean.double(), lse_parts.double())
+    assert_output_close(o, O_ref, "float32 merge with empty parts", max_tol=5e-5, mean_tol=1e-6)
+    assert_lse_close(lse.cpu(), lse_ref, "float32 merge lse with empty parts", tol=5e-5)
+
+
 def test_merge_propagates_nan():
     o_parts = torch.randn((2, 1, 1, 8, 128)).to(torch.bfloat16)
     lse_parts = torch.zeros((2, 1, 1, 8))
@@ -226,7 +268,7 @@ def test_merge_empty_parts_never_leak(S):
     assert_lse_close(lse.cpu()[torch.from_numpy(live)], lse_ref[live], f"merge lse S={S}")
 
 
-@pytest.mark.parametrize("name", ["merge_parts_2", "merge_parts_4", "merge_parts_8"])
+@pytest.mark.parametrize("name", ["merge_parts_2", "merge_parts_4", "merge_parts_8", "merge_parts_4_fp32"])
 def test_full_size_merge_workload_sampled(name):
     """The merge benchmark workloads at full size, in the benchmark's launch
     configuration; the oracle merges sampled rows."""

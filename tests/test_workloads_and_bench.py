@@ -90,6 +90,10 @@ def test_flop_counts_match_closed_forms():
     base = lens.sum() * 32 * 128 * 2 * 2 + 2 * 64 * 32 * 128 * 2
     assert bench.decode_bytes(wd, lens) == base
     assert bench.decode_bytes(wp, lens) == base + 4 * (32 + 512 + 63)
+    # Merge bytes per row: S parts of d values and an lse, plus the merged row and lse.
+    rows = 16 * 16384
+    assert bench.merge_bytes(workloads.WORKLOADS["merge_parts_4"]) == rows * (4 * (256 + 4) + 260)
+    assert bench.merge_bytes(workloads.WORKLOADS["merge_parts_4_fp32"]) == rows * (4 * (512 + 4) + 516)
 
 
 @pytest.mark.parametrize("workload,unit", [("single_head_fp32", "TFLOP/s"), ("paged_kv_decode", "GB/s")])

@@ -199,9 +199,9 @@ def forward_offset(q, k, v, q_offset: int, causal: bool = False, window: int = 0
 def merge(o_parts, lse_parts, out=None, lse=None):
     """Combine S partial results over disjoint key sets into the full attention.
 
-    o_parts: [S, B, H, N, d] (bf16 or fp16, d in {64, 128}); lse_parts:
+    o_parts: [S, B, H, N, d] (bf16, fp16 or float32, d in {64, 128}); lse_parts:
     [S, B, H, N] float32 (-inf marks a part that saw no key for that row).
-    Returns (o [B, H, N, d], lse [B, H, N]).
+    Returns (o [B, H, N, d] in the parts' dtype, lse [B, H, N]).
     """
     _need_cuda(o_parts, lse_parts)
     S, B, H, N, d = o_parts.shape

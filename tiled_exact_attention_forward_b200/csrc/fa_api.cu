@@ -32,7 +32,7 @@ bool sizes_ok(long long B, long long H, long long N) {
 
 extern "C" {
 
-int fa_version(void) { return 103; }
+int fa_version(void) { return 104; }
 
 const char* fa_status_string(fa_status s) {
   switch (s) {
@@ -102,12 +102,13 @@ fa_status fa_merge(const void* o_parts, const float* lse_parts, int S, void* o, 
   if (S < 1 || S > (1 << 16) || !sizes_ok(B, H, N)) return FA_ERR_INVALID;
   if (!aligned(o_parts, 16) || !aligned(o, 16) || !aligned(lse_parts, 4) || (lse && !aligned(lse, 4)))
     return FA_ERR_INVALID;
-  if ((dtype != FA_BF16 && dtype != FA_FP16) || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
+  if ((dtype != FA_BF16 && dtype != FA_FP16 && dtype != FA_FP32) || (d != 64 && d != 128)) return FA_ERR_UNSUPPORTED;
   fa::MergeArgs a{};
   a.o_parts = o_parts; a.lse_parts = lse_parts; a.o = o; a.lse = lse;
   a.rows = static_cast<long long>(B) * H * N;
   a.S = S; a.d = d;
   a.f16 = dtype == FA_FP16;
+  a.f32 = dtype == FA_FP32;
   return from_cuda(fa::launch_merge(a, static_cast<cudaStream_t>(stream)));
 }
 

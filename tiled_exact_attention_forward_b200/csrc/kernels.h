@@ -66,13 +66,14 @@ struct BwdArgs {
 
 // Merge of partial results over disjoint key sets (context parallelism).
 struct MergeArgs {
-  const void* o_parts;     // [S][rows][d] 16-bit, each part normalised
+  const void* o_parts;     // [S][rows][d] 16-bit (or float32 with f32), each part normalised
   const float* lse_parts;  // [S][rows]; -inf marks a part that saw no key
-  void* o;                 // [rows][d] 16-bit
+  void* o;                 // [rows][d], the parts' type
   float* lse;              // [rows], may be null
   long long rows;          // B * H * N
   int S, d;
   int f16;
+  int f32;                 // float32 parts and output
 };
 
 // Decode: keys per split chunk (one CTA each).

@@ -80,6 +80,8 @@ WORKLOADS = {
                  notes="merge of 4 partial results per row, 262144 rows of d = 128"),
         Workload("merge_parts_8", "merge", 1, 8, 16384, 128, BF16, 6, parts=8,
                  notes="merge of 8 partial results per row, 131072 rows of d = 128"),
+        Workload("merge_parts_4_fp32", "merge", 1, 16, 16384, 128, FP32, 6, parts=4,
+                 notes="merge of 4 float32 partial results per row, 262144 rows of d = 128"),
         Workload("context_parallel_causal", "context_parallel", 1, 32, 16384, 128, BF16, 5,
                  causal=True, shards=4, balanced=True,
                  notes="causal forward of a 16K context over 4 ring ranks, each holding sequence "
