@@ -45,6 +45,19 @@ def test_bf16_forward_many_items_per_cta(causal, window):
     assert_lse_close(lse, lse_ref, f"lse many items causal={causal} window={window}")
 
 
+@pytest.mark.parametrize("window", [1, 64, 255, 256, 257, 511, 513, 1100, 5000])
+def test_bf16_forward_causal_window_item_order(window):
+    """Causal sliding windows deal the items whose 256 rows all see a full window
+    first, head by head, then the rest pair-major.  Windows around the 256-row item
+    size move the split point (every item full at window 1, none at a window longer
+    than the sequence); each item must still be computed exactly once."""
+    q, k, v = workloads.forward_inputs(2, 40, 1100, 128, torch.bfloat16, seed=53 + window, device="cpu")
+    o, lse = run_fwd(q.cuda(), k.cuda(), v.cuda(), True, window)
+    O_ref, lse_ref = oracle.attention_forward(q, k, v, None, True, window)
+    assert_output_close(o, O_ref, f"O causal window={window}")
+    assert_lse_close(lse, lse_ref, f"lse causal window={window}")
+
+
 @pytest.mark.parametrize("chunks", [1, 4, 6, 100])
 def test_forward_host_pipelined_over_head_groups(chunks):
     """forward_host splits the 2 x 3 heads into `chunks` groups (clamped to 6) whose
