@@ -259,13 +259,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int s1 = (idx + 1) & 1;
           ok = mbar_wait_warp(smem_u32(&sm.qdo_full[s1]), ((idx + 1) >> 1) & 1, abort_flag);
           if (!ok) break;
-          issue_abT<T>(tmem + T_DP, vd, dod(s1));
-          commit_elect(smem_u32(&sm.dp_full));
+          // S^T of the next tile first (its columns hold dQ until the read-out frees
+          // them): the P/dS warps start on P^T as soon as it lands, and dP^T, needed
+          // only for dS^T, follows it (measured 0.5 % faster than dP^T first).
           ok = mbar_wait_warp(smem_u32(&sm.dq_free), idx & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           issue_abT<T>(tmem + T_S, kd, qd(s1));
           commit_elect(smem_u32(&sm.s_full));
+          issue_abT<T>(tmem + T_DP, vd, dod(s1));
+          commit_elect(smem_u32(&sm.dp_full));
         }
       }
       commit_elect(smem_u32(&sm.acc_done));
