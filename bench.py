@@ -271,6 +271,19 @@ def oracle_sample(w, budget_s=12.0):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+# What the roofline's duration covers, per workload kind, and (for a step of several
+# launches whose dominant kernel can be timed on its own call) that call and its units.
+ROOF_TIMED = {
+    "forward": "the fwd_tc_kernel launch (one per step)",
+    "forward_backward": "one fa_backward call (bwd_pre, bwd_main, bwd_post), timed apart from the forward",
+    "decode": "one fa_decode call (split and combine kernels)",
+    "paged_decode": "one fa_decode_paged call (split and combine kernels)",
+    "merge": "the merge_kernel launch (one per step)",
+    "context_parallel": "the whole ring step (every key-chunk partial and merge)",
+}
+ROOF_CALL = {}  # kind -> (callable, units per call), filled by make_step
+
+
 def make_step(w, dev, rank=0, world=1):
     """Returns (step_fn, e2e_fn, units_per_step, unit, metric, launches_per_step, kernel, sources).
 
@@ -379,6 +392,12 @@ def make_step(w, dev, rank=0, world=1):
         fa.forward(q, k, v, w.causal, w.window, w.scale, out=o, lse=lse)
         if with_bwd:
             fa.backward(q, k, v, o, dO, lse, w.causal, w.window, w.scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    if with_bwd:
+        def bwd_only():
+            fa.backward(q, k, v, o, dO, lse, w.causal, w.window, w.scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+        ROOF_CALL["forward_backward"] = (bwd_only, backward_flops(w) / 1e12)
 
     host_in = [t.cpu().pin_memory() for t in ins]
     outs = [o, lse] + ([dq, dk, dv] if with_bwd else [])
@@ -601,10 +620,21 @@ def run_gpu(args, rank, world, local_rank):
     value = whole_job_rate(units, world, ms)
     e2e_value = whole_job_rate(units, world, e2e_ms)
     hbm, tflops, peak_kind = load_peaks()
+    roof_units, roof_ms = units, ms
+    if w.kind in ROOF_CALL:
+        # The dominant kernel's own call, timed like the steps (L2 flushed between
+        # calls); its inputs are the last timed step's.
+        fn, roof_units = ROOF_CALL[w.kind]
+        roof_ms = float(np.mean(timed_loop(fn, args.steps, 0, flush, stream)))
+        barrier()
+        if dist:
+            roof_ms = max_over_ranks([roof_ms], device=dev)[0]
     if unit == "GB/s":
-        roof = {"bound": "hbm", "achieved": units / (ms / 1e3), "peak": hbm, "unit": "GB/s"}
+        roof = {"bound": "hbm", "achieved": roof_units / (roof_ms / 1e3), "peak": hbm, "unit": "GB/s"}
     else:
-        roof = {"bound": "tensor", "achieved": units / (ms / 1e3), "peak": tflops, "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": roof_units / (roof_ms / 1e3), "peak": tflops, "unit": "TFLOP/s"}
+    roof["timed"] = ROOF_TIMED.get(w.kind, "the step")
+    roof["ms"] = roof_ms
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_kind} ({'copy bandwidth' if unit == 'GB/s' else 'cuBLAS bf16 burst'})"
     roof["kernel"] = kernel
