@@ -28,6 +28,17 @@ namespace mrg {
 
 constexpr int THREADS = 128;
 
+// Streaming 16-byte load: not kept in L1, with a 256-byte L2 fetch granularity (a
+// warp reads 512 contiguous bytes of a part per load).  Measured against plain
+// read-only loads: 2 / 4 / 8 parts 5.5 / 5.2 -> 5.4 / 4.8 -> 5.1-5.2 TB/s.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
 // Conversions between 16-byte words of the parts' type and float32: a word holds
 // 8 elements of a 16-bit type or 4 of float32 (tag F32).
 struct F32 {};
@@ -100,7 +111,7 @@ __global__ void __launch_bounds__(THREADS) merge_kernel(MergeArgs a) {
           l[r][i] = in ? __ldg(a.lse_parts + s * a.rows + row) : -INFINITY;
           const uint4* src = parts + s * part_words + static_cast<size_t>(row) * WPR + sub * NV;
 #pragma unroll
-          for (int k = 0; k < NV; ++k) o[r][i][k] = in ? __ldg(src + k) : make_uint4(0u, 0u, 0u, 0u);
+          for (int k = 0; k < NV; ++k) o[r][i][k] = in ? ld_stream(src + k) : make_uint4(0u, 0u, 0u, 0u);
         }
       }
 #pragma unroll
