@@ -30,7 +30,8 @@ constexpr int THREADS = 128;
 
 // Streaming 16-byte load: not kept in L1, with a 256-byte L2 fetch granularity (a
 // warp reads 512 contiguous bytes of a part per load).  Measured against plain
-// read-only loads: 2 / 4 / 8 parts 5.5 / 5.2 -> 5.4 / 4.8 -> 5.1-5.2 TB/s.
+// read-only loads (TB/s): 2 parts 5.5 either way, 4 parts 5.2 -> 5.4, 8 parts
+// 4.8 -> 5.1-5.2.
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
