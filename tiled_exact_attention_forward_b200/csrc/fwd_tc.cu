@@ -333,7 +333,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------------------------------------------------- Q loader
       // A warp of its own, so the next item's Q tile goes out as soon as the last
       // S MMA of the current item has read the slot, ahead of the K/V stream.  The
-      // item after that has its Q tiles prefetched into L2 meanwhile.
+      // item after that has its Q tiles prefetched into L2 meanwhile (issued after
+      // the current item's loads: at launch that keeps a third item's Q tiles out of
+      // the first DRAM burst, measured 1.5-2 % faster on the 2K causal prefill).
       if (lane == 0) {
         int nq[2] = {0, 0};  // Q tiles loaded so far, per slot
         bool ok = true;
@@ -341,15 +343,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int lin = item_of(k, total);
           if (lin < 0) break;
           const Item it = make_item<OFFSET>(lin, BH, num_pairs, geo);
-          const int lin2 = item_of(k + 1, total);
-          if (lin2 >= 0) {
-            const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
-            for (int t = 0; t < 2; ++t) {
-              if (!active(nx, t)) continue;
-              tma_prefetch_l2_3d(&tm_q, 0, nx.r0[t], nx.bh);
-              tma_prefetch_l2_3d(&tm_q, 64, nx.r0[t], nx.bh);
-            }
-          }
           for (int t = 0; t < 2 && ok; ++t) {
             if (!active(it, t)) continue;
             if (nq[t] > 0) ok = mbar_wait(smem_u32(&sm.q_empty[t]), (nq[t] - 1) & 1, abort_flag);
@@ -359,6 +352,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_3d(smem_u32(sm.q[t]), &tm_q, bar, 0, it.r0[t], it.bh);
             tma_load_3d(smem_u32(sm.q[t]) + HALF_BYTES, &tm_q, bar, 64, it.r0[t], it.bh);
             ++nq[t];
+          }
+          const int lin2 = item_of(k + 1, total);
+          if (ok && lin2 >= 0) {
+            const Item nx = make_item<OFFSET>(lin2, BH, num_pairs, geo);
+            for (int t = 0; t < 2; ++t) {
+              if (!active(nx, t)) continue;
+              tma_prefetch_l2_3d(&tm_q, 0, nx.r0[t], nx.bh);
+              tma_prefetch_l2_3d(&tm_q, 64, nx.r0[t], nx.bh);
+            }
           }
         }
         for (int t = 0; t < 2; ++t)
