@@ -11,21 +11,24 @@
 // Kernels: bwd_pre (D and zeroed fp32 dQ accumulator), bwd_main (below),
 // bwd_post (dQ fp32 -> the inputs' 16-bit type).
 //
-// bwd_main, one CTA per (batch*head, 128-key tile), 576 threads:
+// bwd_main, one CTA per (batch*head, 128-key tile), 576 threads, the CTAs dealt
+// in groups of 8 heads (low key tiles first within a group) so the CTAs in flight
+// keep a few heads' Q, dO and dQ accumulator in L2:
 //   * warp 17 loads K and V once, then (Q_i, dO_i) pairs by TMA into a
 //     two-stage ring;
-//   * warp 16 allocates tensor memory and issues the MMAs from one thread;
+//   * warp 16 allocates tensor memory and issues the MMAs: a warp-uniform loop,
+//     each block of MMAs one asm statement issued by an elected lane;
 //   * warps 0-7 turn S^T, dP^T into P^T and dS^T: warp w handles the key rows
-//     of TMEM lane quarter w%4 and the query columns [64h, 64h + 64),
-//     h = w/4 -- two threads per key row.  P^T and dS^T go back into tensor
-//     memory as 16-bit pairs (operands of the dV and dK MMAs) and dS^T also into
-//     shared memory (operand of the dQ MMA);
+//     of TMEM lane quarter w%4 and, in each 64-query half of the tile, the 32
+//     queries selected by w/4 -- two threads per key row, the halves one after
+//     the other (the first half's dV and dK MMAs run under the second half).
+//     P^T and dS^T go back into tensor memory as 16-bit pairs (operands of the
+//     dV and dK MMAs) and dS^T also into shared memory (operand of the dQ MMA);
 //   * warps 8-15 read dQ_i out of tensor memory (two threads per query row,
-//     64 columns each), stage it in shared memory (the dS buffer, free once
-//     the dQ MMA has read it) and add it into the fp32 accumulator with TMA
-//     bulk reduce-adds, so no per-thread global atomics compete with the
-//     P/dS warps' shared-memory traffic; at the end warps 0-7 write dV and
-//     warps 8-15 write dK.
+//     64 columns each), stage it in the finished (Q_i, dO_i) ring slot and add
+//     it into the fp32 accumulator with TMA bulk reduce-adds, so no per-thread
+//     global atomics compete with the P/dS warps' shared-memory traffic; at the
+//     end warps 0-7 write dV and warps 8-15 write dK.
 // Tensor memory (512 columns): [S^T -> P^T, later dQ_i] [dP^T -> dS^T] [dV] [dK].
 // Keys are the MMA rows of S^T = K Q^T and dP^T = V dO^T, so P^T and dS^T
 // land with keys on lanes -- exactly the A operands dV and dK need.

@@ -29,10 +29,9 @@
 //         warp 13 streams K/V through the ring by TMA, warp 14 loads the Q
 //         tiles (each as soon as its slot frees) and prefetches the next item's
 //         Q tiles into L2.
-//     The MMA warp runs its whole loop warp-uniformly and issues each MMA and
-//     commit from one elected lane; a single thread issues tcgen05.mma barely
-//     faster than the tensor core retires a 128x128x16 step (measured), and a
-//     warp that branches with one active lane issues slower still, so the
+//     The MMA warp runs its whole loop warp-uniformly and issues each 8-MMA
+//     block (one asm statement) and each commit from one elected lane; a warp
+//     that branches with one active lane issues slower (measured), so the
 //     issuer keeps its control flow uniform and its waits and commits few:
 //     per key tile one wait per K/V ring entry (TMA data: no tcgen05 fence),
 //     one P wait per tile, one commit per S and per ring entry.
@@ -40,7 +39,9 @@
 //     epilogue thread and 64 for warpgroup 3 (256*192 + 128*64 + 128*64 =
 //     65536, the block's launch budget of 512 threads x 128).  The host
 //     refuses to launch unless the compiled kernel has exactly that budget.
-//   * Items are dealt to a persistent grid of one CTA per SM, heaviest first.
+//   * Items are dealt to a persistent grid of one CTA per SM, heaviest first
+//     (with a causal window: the full-window items first, head by head, so the
+//     CTAs in flight share a few heads' K/V in L2).
 //     With a causal mask tile 0 of an item ends one key tile before tile 1;
 //     S_0 of the next item's first key tile is then issued at once, so tile
 //     0's softmax warps do not idle across the item boundary.
